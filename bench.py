@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP4 MoE decode layer on B200.
+
+Default workload (the metric's configuration): one token per step through a
+512-expert layer (top-8 + 1 shared, hidden 2560, width 768, MXFP4 weights,
+FP8 activations), rotating over 64 distinct seeded layers (103 GB) so the
+126 MB L2 never holds a repeated layer.  A step = route + experts + combine
+for one token on one layer.  Prints one JSON line.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                  [--workload layer|verify4|stack42]
+
+Under torchrun (N > 1) every rank runs its own independent layer set
+(replicas: the path has no data exchange) and rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+H, I, E, K_TOP, N_SHARED = 2560, 768, 512, 8, 1
+BYTES_PER_EXPERT = 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32   # 3,133,440
+LAYER_BYTES = (E + N_SHARED) * BYTES_PER_EXPERT + E * H * 2
+METRIC = "MoE-layer decode us/token at B=1 and achieved HBM GB/s (% of B200 peak)"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42"])
+    p.add_argument("--layers", type=int, default=64)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- clocks --
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.lines: list[str] = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- layers --
+class Layers:
+    """``n`` seeded E=512 layers resident in HBM, one library handle each."""
+
+    def __init__(self, n, bias=False, max_tokens=4):
+        import torch
+        import mxfp4_expert_layers_b200 as moe
+        import synth.gpu
+        free, _ = torch.cuda.mem_get_info()
+        fit = int((free - (4 << 30)) // LAYER_BYTES)
+        self.requested = n
+        self.n = max(1, min(n, fit))
+        self.bufs, self.handles = [], []
+        nexp = E + N_SHARED
+        for layer in range(self.n):
+            t = {"router_w": torch.empty((E, H), dtype=torch.int16, device="cuda"),
+                 "w13_codes": torch.empty((nexp, 2 * I, H // 2), dtype=torch.uint8, device="cuda"),
+                 "w13_scales": torch.empty((nexp, 2 * I, H // 32), dtype=torch.uint8, device="cuda"),
+                 "w2_codes": torch.empty((nexp, H, I // 2), dtype=torch.uint8, device="cuda"),
+                 "w2_scales": torch.empty((nexp, H, I // 32), dtype=torch.uint8, device="cuda")}
+            synth.gpu.fill_layer(t, 0, layer, E, H, I, N_SHARED)
+            if bias:
+                import synth as S
+                t["router_bias"] = torch.from_numpy(S.zipf_router_bias(0, layer, E)).cuda()
+            self.bufs.append(t)
+            self.handles.append(moe.moe_create(H, I, E, K_TOP, N_SHARED, t, max_tokens))
+        torch.cuda.synchronize()
+
+    def close(self):
+        import mxfp4_expert_layers_b200 as moe
+        for h in self.handles:
+            moe.moe_destroy(h)
+        self.handles = []
+
+
+def alg_bytes(T: int, distinct_routed: int):
+    """Algorithmic bytes of one layer call: weights of the distinct experts
+    touched (routed + shared), the router, activations in/out, and the FP8 h
+    round trip between the two expert kernels."""
+    U = distinct_routed + N_SHARED
+    w13 = U * 2 * I * (H // 2 + H // 32)
+    w2 = U * H * (I // 2 + I // 32)
+    router = E * H * 2
+    act = T * H * 2 * 2
+    hbuf = U * T * I * (4 + 1) * 2
+    gateup = w13 + T * H * 2 + U * T * I * 5
+    return {"layer": w13 + w2 + router + act + hbuf, "gateup": gateup, "down": w2 + U * T * I + T * H * 2,
+            "route": router + T * H * 2}
+
+
+# ----------------------------------------------------------- oracle arm --
+def oracle_sample(n_tokens: int, T: int = 1, budget_s: float = 20.0):
+    """Time the float64 oracle on the host cores on a bounded sample of the
+    same workload: ``n_tokens`` calls of T tokens through layers 0, 1, ...
+    (weights regenerated outside the timed region)."""
+    import synth
+    from oracle import moe as OM
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    times = []
+    for i in range(n_tokens):
+        layer = i % 64
+        x = synth.hidden_states(0, 1000 + i, T, H)
+        lw = OM.LayerWeights(router_w=synth.router_weight(0, layer, E, H), router_bias=None)
+        _, ids, _, _ = OM.route(x, lw, K_TOP)
+        for e in set(ids.ravel().tolist()) | {E}:
+            lw.experts[e] = synth.expert_weights(0, layer, e, H, I)
+        t0 = time.perf_counter()
+        OM.moe_layer(x, lw, E, K_TOP, I, N_SHARED)
+        times.append(time.perf_counter() - t0)
+        if sum(times) > budget_s:
+            break
+    return {"us_per_token": 1e6 * sum(times) / (len(times) * T), "cores": cores,
+            "sample": f"{len(times)} call(s) of {T} token(s), E=512 layers, float64 numpy oracle"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    T = 4 if args.workload == "verify4" else 1
+    for _ in range(args.warmup):
+        oracle_sample(1, T, 1e9)
+    t0 = time.perf_counter()
+    res = oracle_sample(args.steps, T, 1e9)
+    el = time.perf_counter() - t0
+    line = {"metric": METRIC, "value": res["us_per_token"], "unit": "us/token", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args, None),
+            "cpu_baseline": {"value": res["us_per_token"], "unit": "us/token", "cores": res["cores"],
+                             "kind": "oracle", "sample": res["sample"]},
+            "e2e": {"value": res["us_per_token"], "unit": "us/token", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args, layers):
+    n = layers.n if layers is not None else args.layers
+    if args.workload == "layer":
+        w = f"1-token decode, E=512 top-8 + 1 shared, H=2560, I=768, MXFP4 W4A8, {n} rotating layers"
+    elif args.workload == "verify4":
+        w = f"4-token verify call (i.i.d. tokens), E=512 top-8 + 1 shared, {n} rotating layers"
+    else:
+        w = "42-layer decode stack, Zipf(1.1) router bias, residual + RMSNorm chain"
+    c = {"workload": w, "layers_resident": n, "hidden": H, "inter": I, "experts": E, "top_k": K_TOP,
+         "shared": N_SHARED,
+         "l2": "inputs larger than L2: distinct layers rotated (" +
+               f"{n * LAYER_BYTES / 1e9:.1f} GB resident)"}
+    if layers is not None and layers.n < layers.requested:
+        c["note"] = f"only {layers.n} of {layers.requested} layers fit in free HBM"
+    return c
+
+
+# ------------------------------------------------------------- our arm --
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mxfp4_expert_layers_b200 as moe
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    moe.load()
+    hbm_peak, peak_kind = peaks()
+
+    T = 4 if args.workload == "verify4" else 1
+    n_layers = 42 if args.workload == "stack42" else args.layers
+    layers = Layers(n_layers, bias=(args.workload == "stack42"), max_tokens=4)
+    L = layers.n
+    stream = torch.cuda.current_stream()
+    nsteps = args.warmup + args.steps
+
+    # tokens resident in HBM before timing (fresh draw per step)
+    xs_host = np.stack([synth.hidden_states(0, 1000 + 7919 * rank + i, T, H) for i in range(min(nsteps, 512))])
+    xs = torch.from_numpy(xs_host.view(np.int16)).cuda()
+    ids = torch.empty((T, K_TOP), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, K_TOP), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    # stack: residual + normalised input per layer
+    r = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    xin = torch.empty((T, H), dtype=torch.int16, device="cuda")
+
+    def step(i):
+        if args.workload == "stack42":
+            x = xs[i % xs.shape[0]]
+            r.copy_(x)
+            xin.copy_(x)
+            for l in range(L):
+                h = layers.handles[l]
+                moe.moe_route(h, xin, T, ids, wts, None, stream)
+                moe.moe_forward(h, xin, T, ids, wts, y, None, stream)
+                moe.moe_residual_rmsnorm(r, y, xin, T, H, 1e-6, stream)
+        else:
+            h = layers.handles[i % L]
+            x = xs[i % xs.shape[0]]
+            moe.moe_route(h, x, T, ids, wts, None, stream)
+            moe.moe_forward(h, x, T, ids, wts, y, None, stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    prof_handles = layers.handles
+    calls_per_handle = args.steps if args.workload == "stack42" else (args.steps + L - 1) // L
+    for h in prof_handles:
+        moe.moe_profile_begin(h, 3 * calls_per_handle + 3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for i in range(args.warmup, nsteps):
+        step(i)
+    ev1.record(stream)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    kern = {}
+    for h in prof_handles:
+        for name, (t, n) in moe.moe_profile_end(h).items():
+            a, b = kern.get(name, (0.0, 0))
+            kern[name] = (a + t, b + n)
+    clk = clocks.stop()
+
+    # same timed region without per-kernel events (host-overhead check)
+    barrier()
+    ev0.record(stream)
+    for i in range(args.warmup, nsteps):
+        step(i)
+    ev1.record(stream)
+    barrier()
+    ms_noprof = ev0.elapsed_time(ev1)
+
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # distinct experts actually touched (for algorithmic bytes), from the last routing
+    distinct = len(set(ids.cpu().numpy().ravel().tolist()))
+    steps_tokens = args.steps * T
+    per_layer_calls = args.steps * (L if args.workload == "stack42" else 1)
+    if args.workload == "stack42":
+        value = 1e3 * ms / (args.steps * world)          # ms per token of the 42-layer stack -> us
+    else:
+        value = 1e3 * ms / (steps_tokens * world)
+    ab = alg_bytes(T, distinct if T > 1 else K_TOP)
+    layer_us = 1e3 * ms / per_layer_calls
+    gu_ms, gu_n = kern.get("gateup_swiglu", (0.0, 0))
+    dn_ms, dn_n = kern.get("down_combine", (0.0, 0))
+    rt_ms, rt_n = kern.get("route", (0.0, 0))
+    gu_us = 1e3 * gu_ms / max(gu_n, 1)
+    roof = {"bound": "hbm", "kernel": "gateup_swiglu", "achieved": ab["gateup"] / (gu_us * 1e3),
+            "peak": hbm_peak, "unit": "GB/s", "peak_kind": f"{peak_kind} copy bandwidth",
+            "frac": ab["gateup"] / (gu_us * 1e3) / hbm_peak, "traffic": None,
+            "alg_bytes_per_launch": ab["gateup"], "avg_launch_us": gu_us,
+            "other_kernels_us": {"route": 1e3 * rt_ms / max(rt_n, 1), "down_combine": 1e3 * dn_ms / max(dn_n, 1)}}
+    layer_gbs = ab["layer"] / (layer_us * 1e3)
+
+    # e2e through the public API with pinned host buffers
+    xh = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
+    yh = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    xd = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    barrier()
+    ev0.record(stream)
+    for i in range(args.warmup, nsteps):
+        xd.copy_(xh[i % xh.shape[0]], non_blocking=True)
+        if args.workload == "stack42":
+            r.copy_(xd)
+            xin.copy_(xd)
+            for l in range(L):
+                h = layers.handles[l]
+                moe.moe_route(h, xin, T, ids, wts, None, stream)
+                moe.moe_forward(h, xin, T, ids, wts, y, None, stream)
+                moe.moe_residual_rmsnorm(r, y, xin, T, H, 1e-6, stream)
+            yh.copy_(xin, non_blocking=True)
+        else:
+            h = layers.handles[i % L]
+            moe.moe_route(h, xd, T, ids, wts, None, stream)
+            moe.moe_forward(h, xd, T, ids, wts, y, None, stream)
+            yh.copy_(y, non_blocking=True)
+    ev1.record(stream)
+    barrier()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_val = 1e3 * e2e_ms / ((args.steps if args.workload == "stack42" else steps_tokens) * world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res = oracle_sample(30, T, budget_s=20.0)
+        cpu = {"value": res["us_per_token"] * (42 if args.workload == "stack42" else 1),
+               "unit": "us/token", "cores": res["cores"], "kind": "oracle", "sample": res["sample"]}
+
+    launches = per_layer_calls * 3 + (args.steps * L if args.workload == "stack42" else 0)
+    unit = "us/token" if args.workload != "stack42" else "us/token (42-layer stack)"
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e2m1 x e4m3 operands, f32 block sums, f64 accumulation",
+            "data": "synthetic (seeded SplitMix64 weights, Irwin-Hall normals)",
+            "config": workload_config(args, layers),
+            "layer_us": layer_us, "layer_gbs": layer_gbs, "layer_frac_of_peak": layer_gbs / hbm_peak,
+            "layer_frac_of_8tbs": layer_gbs / 8000.0, "alg_bytes_per_layer": ab["layer"],
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": T * H * 2,
+                    "d2h_bytes_per_step": T * H * 2},
+            "gpu_launches": launches, "clocks": clk, "ms_per_step_without_profiling": ms_noprof / args.steps}
+    if args.workload == "stack42":
+        line["stack_tokens_per_s"] = 1e6 / value
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layers.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * mxfp4_moe.h -- C ABI of the MXFP4 mixture-of-experts decode layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources: "NVIDIA 在单台 DGX Spark 上叠加三项优化，Ling-3.0-flash 的
+ * MoE 推理吞吐提升 42.5%" (tanhow.com), section "Ling 3.0 是什么" sparse-MoE
+ * bullet: each MoE layer routes a token to 8 of 512 routed experts plus 1
+ * shared expert; section "三项优化是什么？" item 1: experts of width 768;
+ * item 2: LM head 157,184 x 2,560, hence hidden 2560; section
+ * "为什么 DGX Spark 上的 MoE 解码是内存受限的？": decode is weight-read bound
+ * and runs the W4A8 recipe; devotd.net retelling, section 2: MXFP4 is a
+ * blocked 4-bit float format):
+ *
+ *   logits  l[t,e] = f32( sum_k x[t,k] W_r[e,k] ) (+ b[e])     float64 sum
+ *   ids     top_k experts by descending logit, ties -> lower index
+ *   w       softmax over the selected logits (= softmax, keep top_k, renormalise)
+ *   xq, xs  FP8 E4M3 codes of x / xs, xs = amax(|x_t|) / 448 (one per token)
+ *   g, u    MXFP4 gate / up GEMV on xq, times xs
+ *   h       silu(g) * u, re-quantised to FP8 per (token, expert): qh, sh
+ *   y[t]    bf16( sum_i w[t,i] Down_{ids[t,i]}(qh) sh + sum_s Down_shared_s(qh) sh )
+ *
+ * MXFP4 (OCP Microscaling Formats v1.0): 32 consecutive elements along K
+ * (the input dimension of a matrix) share one E8M0 scale 2^(e-127); each
+ * element is a 4-bit E2M1 code (bit 3 sign, 2 exponent bits, 1 mantissa
+ * bit).  Two codes per byte, element 2j in the low nibble of byte j.
+ *
+ * Conventions of every entry point:
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *    the library never frees them and never copies weights.  Every device
+ *    pointer must be 16-byte aligned.
+ *  - Work is enqueued on the given stream; no call synchronises the host
+ *    except moe_create, moe_destroy and moe_device_error.
+ *  - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Nothing throws
+ *    or aborts across the ABI.  moe_strerror() names a code.
+ *  - A handle holds one workspace and is not safe for concurrent use from
+ *    several streams or threads.
+ */
+#ifndef MXFP4_MOE_H
+#define MXFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_ARG (-1)         /* null pointer, T <= 0, T > max_tokens, ...  */
+#define MOE_ERR_SHAPE (-2)       /* hidden/inter not multiples of 32, top_k, E  */
+#define MOE_ERR_ALIGN (-3)       /* a pointer is not 16-byte aligned           */
+#define MOE_ERR_CUDA (-4)        /* a CUDA call or launch failed               */
+#define MOE_ERR_TIMEOUT (-5)     /* a bounded device-side wait gave up          */
+#define MOE_ERR_UNSUPPORTED (-6) /* size outside what this build implements    */
+#define MOE_ERR_DEVICE (-7)      /* device-side input check failed (bad ids)   */
+
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 8
+#define MOE_MAX_SHARED 2
+#define MOE_GEMV_MAX_TOKENS 4    /* T above this takes the grouped-GEMM path  */
+
+typedef struct moe_handle_s* moe_handle;
+
+typedef struct {
+  int32_t hidden;     /* H, multiple of 64, <= 16384 (2560)               */
+  int32_t inter;      /* I, expert width, multiple of 64, <= 4096 (768)   */
+  int32_t n_experts;  /* E routed experts, 1..512                          */
+  int32_t top_k;      /* experts per token, 1..8 and <= E                  */
+  int32_t n_shared;   /* shared experts, 0..2, added with weight 1         */
+} moe_config;
+
+/* All device pointers, borrowed: they must stay valid while the handle is
+ * used.  Expert arrays hold the routed experts 0..E-1 followed by the shared
+ * experts E..E+n_shared-1, each expert contiguous:
+ *   w13_codes  [E+S][2I][H/2]  rows 0..I-1 gate, rows I..2I-1 up (uint8)
+ *   w13_scales [E+S][2I][H/32] E8M0 exponents (uint8)
+ *   w2_codes   [E+S][H][I/2]   down projection
+ *   w2_scales  [E+S][H][I/32]
+ *   router_w   [E][H]          bfloat16 bit patterns (uint16)
+ *   router_bias[E]             float32, or NULL for no bias
+ * E8M0 exponent 255 (NaN) is not supported. */
+typedef struct {
+  const uint16_t* router_w;
+  const float* router_bias;
+  const uint8_t* w13_codes;
+  const uint8_t* w13_scales;
+  const uint8_t* w2_codes;
+  const uint8_t* w2_scales;
+} moe_weights;
+
+/* Optional debug outputs of moe_forward (device pointers, each may be NULL):
+ *   xq [T][H] FP8 codes of x, xs [T] their scales,
+ *   h  [T][top_k+n_shared][I] float32 SwiGLU outputs,
+ *   qh [T][top_k+n_shared][I] FP8 codes of h, sh [T][top_k+n_shared] scales,
+ * slots in ids order, shared experts last. */
+typedef struct {
+  uint8_t* xq;
+  float* xs;
+  float* h;
+  uint8_t* qh;
+  float* sh;
+} moe_debug;
+
+/* Create a handle for one layer.  Validates the configuration (MOE_ERR_SHAPE)
+ * and pointer alignment (MOE_ERR_ALIGN), then allocates a workspace sized for
+ * max_tokens tokens per call (MOE_ERR_CUDA if that fails).  The weights are
+ * borrowed, not copied.  *out is set only on success. */
+int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens,
+               moe_handle* out);
+
+/* Route T tokens: x [T][H] bfloat16 (device) -> topk_ids [T][top_k] int32
+ * (descending logit, ties to the lower expert index), topk_w [T][top_k]
+ * float32 (renormalised softmax weights, sum 1), expert_counts [E] int32
+ * (tokens per routed expert; may be NULL).  One kernel launch.
+ * Errors: MOE_ERR_ARG for null pointers or T outside 1..max_tokens. */
+int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
+              int32_t* expert_counts, cudaStream_t stream);
+
+/* Run the experts of T tokens and combine: x [T][H] bfloat16 (device), the
+ * routing from moe_route (or any ids in 0..E-1 and weights the caller
+ * chooses), y [T][H] bfloat16 (device, written).  dbg may be NULL.
+ * T <= MOE_GEMV_MAX_TOKENS runs the split-K GEMV path; larger T runs the
+ * dispatch + grouped-GEMM path.  Ids outside 0..E-1 are skipped and recorded
+ * (see moe_device_error).  Errors: MOE_ERR_ARG, MOE_ERR_UNSUPPORTED. */
+int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
+                const float* topk_w, uint16_t* y, const moe_debug* dbg,
+                cudaStream_t stream);
+
+/* Synchronise the stream and report (then clear) device-side errors
+ * recorded by earlier calls: MOE_ERR_DEVICE for out-of-range expert ids,
+ * MOE_ERR_TIMEOUT if a bounded wait inside a kernel gave up. */
+int moe_device_error(moe_handle h, cudaStream_t stream);
+
+/* Which kernel path the last moe_forward on this handle launched:
+ * 1 = GEMV (T <= MOE_GEMV_MAX_TOKENS), 2 = grouped GEMM, 0 = none yet. */
+int moe_last_path(moe_handle h);
+
+/* Per-kernel timing.  moe_profile_begin(h, n) makes the following calls on
+ * this handle record a CUDA event pair around each kernel they launch (up to
+ * n launches; further launches are not timed).  moe_profile_end synchronises,
+ * writes for each kernel id -- 0 router, 1 gate/up + SwiGLU, 2 down + combine,
+ * 3 reserved -- the summed milliseconds to ms[id] and the timed launches to
+ * launches[id] (arrays of MOE_PROFILE_KERNELS entries), and stops recording.
+ * The events are recorded on the stream each kernel runs on.  Errors:
+ * MOE_ERR_ARG, MOE_ERR_CUDA. */
+#define MOE_PROFILE_KERNELS 4
+int moe_profile_begin(moe_handle h, int max_launches);
+int moe_profile_end(moe_handle h, float* ms, int* launches);
+
+/* Free the workspace (synchronises the device first).  NULL is accepted. */
+int moe_destroy(moe_handle h);
+
+/* Static text for a return code. */
+const char* moe_strerror(int code);
+
+/* Per-row FP8 E4M3 quantisation, the activation step of the W4A8 recipe
+ * (tanhow.com retelling, "为什么 DGX Spark 上的 MoE 解码是内存受限的？";
+ * devotd.net retelling, section 2: 8-bit activations) as a standalone call:
+ * v [rows][cols] float32 (device) -> q [rows][cols] E4M3 codes (uint8) and
+ * s [rows] float32 with s = amax/448 (IEEE division; 1 if the row is all
+ * zero) and q = E4M3(v / s), round to nearest even, saturating to +-448.
+ * The same encoder moe_forward applies to x and to the SwiGLU output.
+ * Errors: MOE_ERR_ARG (null pointer, rows or cols < 1). */
+int moe_quantize_fp8(const float* v, int rows, int cols, uint8_t* q, float* s,
+                     cudaStream_t stream);
+
+/* Harness step for chained layers (not part of the MoE layer):
+ * r[t] = bf16(r[t] + y[t]) in place, then
+ * x_next[t] = bf16( r[t] / sqrt(mean_k r[t,k]^2 + eps) ).  All [T][H]
+ * bfloat16 device arrays.  Returns MOE_ERR_ARG on bad arguments. */
+int moe_residual_rmsnorm(uint16_t* r, const uint16_t* y, uint16_t* x_next, int T, int H,
+                         float eps, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXFP4_MOE_H */

@@ -1,0 +1,175 @@
+"""MXFP4 mixture-of-experts decode layer for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libmxfp4moe.so`` (CUDA kernels behind the C ABI of
+``include/mxfp4_moe.h``).  This package is a thin ctypes binding with the
+same entry-point names: it converts arguments (torch tensors -> device
+pointers, CUDA streams -> handles) and raises :class:`MoEError` on a
+non-zero return code.  There is no other implementation behind it: if the
+library cannot be loaded every call fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxfp4moe.so")
+
+MOE_OK = 0
+MOE_ERR_ARG = -1
+MOE_ERR_SHAPE = -2
+MOE_ERR_ALIGN = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+MOE_ERR_UNSUPPORTED = -6
+MOE_ERR_DEVICE = -7
+MOE_GEMV_MAX_TOKENS = 4
+
+EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
+           "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
+           "moe_profile_begin", "moe_profile_end")
+MOE_PROFILE_KERNELS = 4
+KERNEL_NAMES = ("route", "gateup_swiglu", "down_combine", "reserved")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} ({code})")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("w13_codes", ctypes.c_void_p), ("w13_scales", ctypes.c_void_p),
+                ("w2_codes", ctypes.c_void_p), ("w2_scales", ctypes.c_void_p)]
+
+
+class moe_debug(ctypes.Structure):
+    _fields_ = [("xq", ctypes.c_void_p), ("xs", ctypes.c_void_p), ("h", ctypes.c_void_p),
+                ("qh", ctypes.c_void_p), ("sh", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises OSError if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    L = ctypes.CDLL(path)
+    p, i = ctypes.c_void_p, ctypes.c_int
+    L.moe_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), i,
+                             ctypes.POINTER(p)]
+    L.moe_route.argtypes = [p, p, i, p, p, p, p]
+    L.moe_forward.argtypes = [p, p, i, p, p, p, ctypes.POINTER(moe_debug), p]
+    L.moe_device_error.argtypes = [p, p]
+    L.moe_last_path.argtypes = [p]
+    L.moe_destroy.argtypes = [p]
+    L.moe_strerror.argtypes = [i]
+    L.moe_strerror.restype = ctypes.c_char_p
+    L.moe_profile_begin.argtypes = [p, i]
+    L.moe_profile_end.argtypes = [p, p, p]
+    L.moe_quantize_fp8.argtypes = [p, i, i, p, p, p]
+    L.moe_residual_rmsnorm.argtypes = [p, p, p, i, i, ctypes.c_float, p]
+    for name in EXPORTS:
+        if name != "moe_strerror":
+            getattr(L, name).restype = i
+    _lib = L
+    return L
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int, where: str) -> int:
+    if rc != MOE_OK:
+        raise MoEError(rc, where)
+    return rc
+
+
+def strerror(code: int) -> str:
+    return load().moe_strerror(code).decode()
+
+
+moe_strerror = strerror
+
+
+def moe_create(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
+               weights: dict, max_tokens: int) -> int:
+    """Returns an opaque handle.  ``weights`` maps the moe_weights field names
+    to CUDA tensors (``router_bias`` may be None)."""
+    cfg = moe_config(hidden, inter, n_experts, top_k, n_shared)
+    w = moe_weights(*[_ptr(weights.get(f)) for f, _ in moe_weights._fields_])
+    h = ctypes.c_void_p()
+    _check(load().moe_create(ctypes.byref(cfg), ctypes.byref(w), max_tokens, ctypes.byref(h)),
+           "moe_create")
+    return h.value
+
+
+def moe_route(handle: int, x, T: int, topk_ids, topk_w, expert_counts=None, stream=None) -> None:
+    _check(load().moe_route(handle, _ptr(x), T, _ptr(topk_ids), _ptr(topk_w),
+                            _ptr(expert_counts), _stream(stream)), "moe_route")
+
+
+def moe_forward(handle: int, x, T: int, topk_ids, topk_w, y, dbg: dict | None = None,
+                stream=None) -> None:
+    d = None
+    if dbg:
+        d = ctypes.byref(moe_debug(*[_ptr(dbg.get(f)) for f, _ in moe_debug._fields_]))
+    _check(load().moe_forward(handle, _ptr(x), T, _ptr(topk_ids), _ptr(topk_w), _ptr(y), d,
+                              _stream(stream)), "moe_forward")
+
+
+def moe_device_error(handle: int, stream=None) -> int:
+    """Returns the code (does not raise) so callers can test for errors."""
+    return load().moe_device_error(handle, _stream(stream))
+
+
+def moe_last_path(handle: int) -> int:
+    return load().moe_last_path(handle)
+
+
+def moe_destroy(handle: int) -> None:
+    _check(load().moe_destroy(handle), "moe_destroy")
+
+
+def moe_profile_begin(handle: int, max_launches: int) -> None:
+    _check(load().moe_profile_begin(handle, max_launches), "moe_profile_begin")
+
+
+def moe_profile_end(handle: int) -> dict:
+    """Returns ``{kernel name: (total ms, launches)}``."""
+    ms = (ctypes.c_float * MOE_PROFILE_KERNELS)()
+    n = (ctypes.c_int * MOE_PROFILE_KERNELS)()
+    _check(load().moe_profile_end(handle, ms, n), "moe_profile_end")
+    return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(MOE_PROFILE_KERNELS)}
+
+
+def moe_quantize_fp8(v, rows: int, cols: int, q, s, stream=None) -> None:
+    _check(load().moe_quantize_fp8(_ptr(v), rows, cols, _ptr(q), _ptr(s), _stream(stream)),
+           "moe_quantize_fp8")
+
+
+def moe_residual_rmsnorm(r, y, x_next, T: int, H: int, eps: float = 1e-6, stream=None) -> None:
+    _check(load().moe_residual_rmsnorm(_ptr(r), _ptr(y), _ptr(x_next), T, H, eps, _stream(stream)),
+           "moe_residual_rmsnorm")

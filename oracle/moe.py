@@ -198,3 +198,20 @@ def down_replay(ex: dict, qh: np.ndarray, sh: np.float32) -> np.ndarray:
     """The down GEMV alone on given FP8 activations (used to check the down
     step in isolation from the re-quantisation of h)."""
     return mxfp4_matvec(ex["w2_codes"], ex["w2_scales"], qh, sh)
+
+
+# ------------------------------------------------- chained-layer harness --
+
+def residual_rmsnorm(r_bf16: np.ndarray, y_bf16: np.ndarray, eps: float = 1e-6):
+    """Harness step between chained layers (not part of the MoE layer; the
+    pages do not describe the stack's normalisation -- plain reading: residual
+    add, RMS normalisation without a learned weight):
+    ``r = bf16(r + y)``; ``x = bf16( r / sqrt(mean(r**2) + eps) )`` with the
+    sum, mean, square root and division in float64."""
+    r = f64_to_bf16(bf16_to_f64(r_bf16) + bf16_to_f64(y_bf16))
+    rv = bf16_to_f64(r)
+    ms = np.zeros(rv.shape[0])
+    for k in range(rv.shape[1]):
+        ms += rv[:, k] * rv[:, k]
+    den = np.sqrt(ms / rv.shape[1] + np.float64(np.float32(eps)))
+    return r, f64_to_bf16(rv / den[:, None])

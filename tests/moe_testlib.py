@@ -1,0 +1,147 @@
+"""Helpers of the GPU parity tests: build a layer on the device (seeded
+generator), call the library through its C ABI, and build the matching host
+view for the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import mxfp4_expert_layers_b200 as moe
+import synth
+import synth.gpu
+from oracle import formats as OF
+from oracle import moe as OM
+
+H0, I0 = 2560, 768
+REL_L2 = 2e-3          # output tolerance of the layer (relative L2)
+MAX_ABS = 1e-2         # max |delta| <= MAX_ABS * max |ref|
+
+
+class LazyExperts(dict):
+    """Expert arrays regenerated on the host on first use."""
+
+    def __init__(self, seed, layer, H, I):
+        super().__init__()
+        self.args = (seed, layer, H, I)
+
+    def __missing__(self, e):
+        seed, layer, H, I = self.args
+        v = synth.expert_weights(seed, layer, int(e), H, I)
+        self[e] = v
+        return v
+
+
+def to_dev_u16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+class GpuLayer:
+    def __init__(self, seed, layer, E, H=H0, I=I0, k=8, n_shared=1, bias=False, max_tokens=4,
+                 fill="gpu", weights=None):
+        self.seed, self.layer, self.E, self.H, self.I, self.k, self.S = seed, layer, E, H, I, k, n_shared
+        n = E + n_shared
+        dev = "cuda"
+        if weights is None:
+            self.t = {
+                "router_w": torch.empty((E, H), dtype=torch.int16, device=dev),
+                "w13_codes": torch.empty((n, 2 * I, H // 2), dtype=torch.uint8, device=dev),
+                "w13_scales": torch.empty((n, 2 * I, H // 32), dtype=torch.uint8, device=dev),
+                "w2_codes": torch.empty((n, H, I // 2), dtype=torch.uint8, device=dev),
+                "w2_scales": torch.empty((n, H, I // 32), dtype=torch.uint8, device=dev),
+            }
+            if fill == "gpu":
+                synth.gpu.fill_layer(self.t, seed, layer, E, H, I, n_shared)
+            else:
+                lw = synth.layer_weights(seed, layer, E, H, I, n_shared)
+                self.t["router_w"].copy_(to_dev_u16(lw["router_w"]))
+                for key in ("w13_codes", "w13_scales", "w2_codes", "w2_scales"):
+                    self.t[key].copy_(to_dev(lw[key]))
+            self.host = OM.LayerWeights(router_w=synth.router_weight(seed, layer, E, H), router_bias=None,
+                                        experts=LazyExperts(seed, layer, H, I))
+        else:  # explicit host arrays (edge-case tests)
+            self.t = {"router_w": to_dev_u16(weights["router_w"])}
+            for key in ("w13_codes", "w13_scales", "w2_codes", "w2_scales"):
+                self.t[key] = to_dev(weights[key])
+            ex = {e: {key: weights[key][e] for key in ("w13_codes", "w13_scales", "w2_codes", "w2_scales")}
+                  for e in range(n)}
+            self.host = OM.LayerWeights(router_w=weights["router_w"], router_bias=None, experts=ex)
+        if bias is not False:
+            b = synth.zipf_router_bias(seed, layer, E) if bias is True else np.asarray(bias, np.float32)
+            self.t["router_bias"] = to_dev(b)
+            self.host.router_bias = b
+        torch.cuda.synchronize()
+        self.handle = moe.moe_create(H, I, E, k, n_shared, self.t, max_tokens)
+
+    def close(self):
+        if self.handle:
+            moe.moe_destroy(self.handle)
+            self.handle = None
+
+    def route(self, x_dev, T):
+        ids = torch.empty((T, self.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, self.k), dtype=torch.float32, device="cuda")
+        counts = torch.empty((self.E,), dtype=torch.int32, device="cuda")
+        moe.moe_route(self.handle, x_dev, T, ids, w, counts, torch.cuda.current_stream())
+        return ids, w, counts
+
+    def forward(self, x_dev, T, ids, w, debug=True):
+        S = self.k + self.S
+        y = torch.empty((T, self.H), dtype=torch.int16, device="cuda")
+        dbg = None
+        if debug:
+            dbg = {"xq": torch.empty((T, self.H), dtype=torch.uint8, device="cuda"),
+                   "xs": torch.empty((T,), dtype=torch.float32, device="cuda"),
+                   "h": torch.empty((T, S, self.I), dtype=torch.float32, device="cuda"),
+                   "qh": torch.empty((T, S, self.I), dtype=torch.uint8, device="cuda"),
+                   "sh": torch.empty((T, S), dtype=torch.float32, device="cuda")}
+        moe.moe_forward(self.handle, x_dev, T, ids, w, y, dbg, torch.cuda.current_stream())
+        return y, dbg
+
+
+def check_route(g_ids, g_w, g_counts, ref):
+    ids = g_ids.cpu().numpy()
+    assert np.array_equal(ids, ref["ids"]), (ids, ref["ids"])
+    if g_counts is not None:
+        assert np.array_equal(g_counts.cpu().numpy(), ref["counts"])
+    w = g_w.cpu().numpy()
+    assert np.allclose(w, ref["w"], rtol=1e-6, atol=1e-7)
+
+
+def legit_fp8_flip(v_ref: float, code_a: int, code_b: int) -> bool:
+    """Two adjacent codes are both acceptable when the exact value sits within
+    1e-6 (relative) of the midpoint between them."""
+    va, vb = float(OF.e4m3_value(code_a)), float(OF.e4m3_value(code_b))
+    return abs(abs(va) - abs(vb)) > 0 and abs(v_ref - (va + vb) / 2) <= 1e-6 * max(abs(v_ref), 1e-30)
+
+
+def check_forward(y_dev, dbg, ref, exact_frac=0.999):
+    """Tolerance of the layer, plus the stronger bit-level checks the exact
+    arithmetic of the GEMV path allows."""
+    yg = OF.bf16_to_f64(u16(y_dev))
+    yr = OF.bf16_to_f64(ref["y"])
+    rel = np.linalg.norm(yg - yr) / max(np.linalg.norm(yr), 1e-300)
+    mx = np.abs(yg - yr).max() / max(np.abs(yr).max(), 1e-300)
+    assert rel <= REL_L2 and mx <= MAX_ABS, (rel, mx)
+    stats = {"rel_l2": rel, "max_rel": mx, "y_exact": float(np.mean(u16(y_dev) == ref["y"]))}
+    if dbg is not None:
+        assert np.array_equal(dbg["xq"].cpu().numpy(), ref["xq"])
+        assert np.array_equal(dbg["xs"].cpu().numpy(), ref["xs"])
+        qg = dbg["qh"].cpu().numpy()
+        bad = np.argwhere(qg != ref["qh"])
+        for t, s, j in bad:
+            v = float(ref["h"][t, s, j]) / float(ref["sh"][t, s])
+            assert legit_fp8_flip(v, int(qg[t, s, j]), int(ref["qh"][t, s, j])), (t, s, j)
+        stats["qh_flips"] = len(bad)
+        stats["h_exact"] = float(np.mean(dbg["h"].cpu().numpy() == ref["h"]))
+        if len(bad) == 0:
+            assert np.array_equal(dbg["sh"].cpu().numpy(), ref["sh"])
+    assert stats["y_exact"] >= exact_frac, stats
+    return stats

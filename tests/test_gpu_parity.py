@@ -1,0 +1,286 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle on
+the same seeded inputs.  Bars: expert ids and counts bit-exact, FP8
+activation bytes bit-exact, BF16 outputs within relative L2 <= 2e-3 and
+max |delta| <= 1e-2 * max |ref|; the GEMV path's exact block arithmetic
+also gives bit-exact FP8 codes of h and (almost always) bit-exact outputs,
+which the tests check too."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_expert_layers_b200 as moe
+import synth
+from oracle import formats as OF
+from oracle import moe as OM
+
+from moe_testlib import (GpuLayer, check_forward, check_route, to_dev, to_dev_u16, u16,
+                         H0, I0)
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU collection
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+
+def _oracle(layer: GpuLayer, x_bits):
+    return OM.moe_layer(x_bits, layer.host, layer.E, layer.k, layer.I, layer.S)
+
+
+def _run(layer: GpuLayer, x_bits, debug=True):
+    T = x_bits.shape[0]
+    xd = to_dev_u16(x_bits)
+    ids, w, counts = layer.route(xd, T)
+    y, dbg = layer.forward(xd, T, ids, w, debug)
+    torch.cuda.synchronize()
+    assert moe.moe_device_error(layer.handle) == moe.MOE_OK
+    return ids, w, counts, y, dbg
+
+
+# ------------------------------------------------------------ generators --
+
+def test_gpu_fill_matches_host_generator():
+    E, H, I = 16, 256, 128
+    L = GpuLayer(5, 3, E, H, I, k=4, fill="gpu")
+    try:
+        assert np.array_equal(u16(L.t["router_w"]), synth.router_weight(5, 3, E, H))
+        for e in (0, 7, E):                          # includes the shared expert
+            ref = synth.expert_weights(5, 3, e, H, I)
+            for key in ref:
+                assert np.array_equal(L.t[key][e].cpu().numpy(), ref[key]), (e, key)
+    finally:
+        L.close()
+
+
+# ----------------------------------------------------------------- FP8 ---
+
+def _structured_fp32():
+    hi = np.arange(1 << 16, dtype=np.uint32) << np.uint32(16)
+    lows = np.array([0, 1, 0x7FFF, 0x8000, 0x8001, 0xFFFF, 0x1234, 0xC000], dtype=np.uint32)
+    pats = (hi[:, None] | lows[None, :]).ravel()
+    v = pats.view(np.float32)
+    return v[np.isfinite(v) & (np.abs(v) <= 448.0)]
+
+
+def test_gpu_fp8_encoder_matches_oracle():
+    """Rows [v, 448]: the scale is exactly 1, so the codes are the plain
+    encoder on every structured float32 pattern of magnitude <= 448 (every
+    sign/exponent/top-7-mantissa combination with boundary low bits), plus
+    every exact midpoint between adjacent E4M3 values and its neighbours."""
+    v = _structured_fp32()
+    vals = np.unique(np.abs(OF.e4m3_value(np.arange(0x7F))))
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    extra = np.concatenate([mids, np.nextafter(mids, np.float32(0)),
+                            np.nextafter(mids, np.float32(np.inf)), vals.astype(np.float32)])
+    v = np.concatenate([v, extra, -extra]).astype(np.float32)
+    rows = np.stack([v, np.full_like(v, 448.0)], axis=1)
+    q = torch.empty(rows.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows.shape[0], dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8(to_dev(rows), rows.shape[0], 2, q, s)
+    torch.cuda.synchronize()
+    assert np.all(s.cpu().numpy() == 1.0)
+    got = q.cpu().numpy()[:, 0]
+    ref = OF.e4m3_encode(v)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(v[i]), int(got[i]), int(ref[i])) for i in bad[:8]]
+
+
+def test_gpu_quantize_rows_matches_oracle():
+    rng = np.random.default_rng(0)
+    v = (rng.standard_normal((37, 1000)) * rng.uniform(1e-3, 1e3, (37, 1))).astype(np.float32)
+    v[3] = 0.0
+    v[5, :] = -0.0
+    q = torch.empty(v.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(v.shape[0], dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8(to_dev(v), v.shape[0], v.shape[1], q, s)
+    rq, rs = OM.quantize_fp8(v)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy(), rs)
+
+
+# --------------------------------------------------------------- routing --
+
+@pytest.mark.parametrize("E,T,bias", [(32, 1, False), (512, 1, False), (512, 4, False),
+                                      (512, 4, True), (512, 37, True)])
+def test_gpu_route_matches_oracle(E, T, bias):
+    L = GpuLayer(0, 0, E, k=8, bias=bias, max_tokens=max(T, 4))
+    try:
+        x = synth.hidden_states(0, 1000 + T, T, H0)
+        ids, w, counts = L.route(to_dev_u16(x), T)
+        l, rid, rw, rc = OM.route(x, L.host, 8)
+        check_route(ids, w, counts, {"ids": rid, "w": rw, "counts": rc})
+        assert np.all(np.abs(w.cpu().numpy().astype(np.float64).sum(1) - 1) <= 1e-6)
+    finally:
+        L.close()
+
+
+def test_gpu_route_ties_go_to_lower_index():
+    E, H, I = 16, 128, 64
+    lw = synth.layer_weights(1, 0, E, H, I)
+    lw["router_w"][9] = lw["router_w"][2]          # identical rows -> identical logits
+    lw["router_w"][14] = lw["router_w"][2]
+    L = GpuLayer(1, 0, E, H, I, k=4, weights=lw)
+    try:
+        x = synth.hidden_states(1, 0, 4, H)
+        ids, w, counts = L.route(to_dev_u16(x), 4)
+        l, rid, rw, rc = OM.route(x, L.host, 4)
+        check_route(ids, w, counts, {"ids": rid, "w": rw, "counts": rc})
+        for t in range(4):
+            row = ids[t].tolist()
+            for a, b in ((2, 9), (2, 14), (9, 14)):
+                if a in row and b in row:
+                    assert row.index(a) < row.index(b)
+    finally:
+        L.close()
+
+
+# ------------------------------------------------------------- forward --
+
+@pytest.mark.parametrize("n_shared", [0, 1, 2])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_gpu_forward_small_shapes(T, n_shared):
+    E, H, I, k = 8, 128, 64, 2
+    L = GpuLayer(2, T, E, H, I, k=k, n_shared=n_shared, fill="host")
+    try:
+        for step in range(3):
+            x = synth.hidden_states(2, 10 * T + step, T, H)
+            ids, w, counts, y, dbg = _run(L, x)
+            ref = _oracle(L, x)
+            check_route(ids, w, counts, ref)
+            check_forward(y, dbg, ref)
+    finally:
+        L.close()
+
+
+def test_gpu_forward_config0_single_token():
+    """One token, E = 32 routed top-8 + 1 shared, H 2560, I 768, seed 0."""
+    L = GpuLayer(0, 0, 32)
+    try:
+        for step in range(4):
+            x = synth.hidden_states(0, step, 1, H0)
+            ids, w, counts, y, dbg = _run(L, x)
+            ref = _oracle(L, x)
+            check_route(ids, w, counts, ref)
+            st = check_forward(y, dbg, ref)
+            assert st["qh_flips"] == 0 and st["h_exact"] == 1.0, st
+    finally:
+        L.close()
+
+
+def test_gpu_forward_config1_full_layer():
+    """E = 512 (the 1.6 GB layer) at full size; tokens one at a time."""
+    for layer in (0, 1):
+        L = GpuLayer(0, layer, 512)
+        try:
+            for step in range(3):
+                x = synth.hidden_states(0, 1000 + 10 * layer + step, 1, H0)
+                ids, w, counts, y, dbg = _run(L, x)
+                ref = _oracle(L, x)
+                check_route(ids, w, counts, ref)
+                check_forward(y, dbg, ref)
+                # replay: the oracle's down + combine on the GPU's own FP8 h
+                qh, sh = dbg["qh"].cpu().numpy()[0], dbg["sh"].cpu().numpy()[0]
+                slots = [(int(e), float(p)) for e, p in zip(ref["ids"][0], ref["w"][0])] + [(512, 1.0)]
+                y64 = np.zeros(H0)
+                for si, (e, p) in enumerate(slots):
+                    y64 += p * OM.down_replay(L.host.experts[e], qh[si], sh[si])
+                assert np.array_equal(OF.f64_to_bf16(y64), u16(y)[0])
+        finally:
+            L.close()
+
+
+@pytest.mark.parametrize("kind", ["iid", "clustered"])
+def test_gpu_forward_config2_four_tokens(kind):
+    """Speculative verify: 4 tokens through the E = 512 layer in one call,
+    i.i.d. or 4 copies of one vector + N(0, 0.1^2) noise; also equal to 4
+    single-token calls."""
+    L = GpuLayer(0, 2, 512)
+    try:
+        if kind == "iid":
+            x = synth.hidden_states(0, 2000, 4, H0)
+        else:
+            x = synth.hidden_states_clustered(0, 2001, 4, H0)
+        ids, w, counts, y, dbg = _run(L, x)
+        ref = _oracle(L, x)
+        check_route(ids, w, counts, ref)
+        check_forward(y, dbg, ref)
+        distinct = len(set(ref["ids"].ravel().tolist()))
+        assert distinct <= 32
+        for t in range(4):
+            i1, w1, c1, y1, _ = _run(L, x[t:t + 1], debug=False)
+            assert np.array_equal(i1.cpu().numpy()[0], ids.cpu().numpy()[t])
+            assert np.array_equal(u16(y1)[0], u16(y)[t])
+    finally:
+        L.close()
+
+
+# ------------------------------------------------------------ edge cases --
+
+def test_gpu_zero_input_and_zero_weights():
+    E, H, I = 8, 128, 64
+    L = GpuLayer(3, 0, E, H, I, k=2, fill="host")
+    try:
+        x = np.zeros((2, H), np.uint16)
+        ids, w, counts, y, dbg = _run(L, x)
+        assert not u16(y).any()
+        assert np.all(dbg["xs"].cpu().numpy() == 1.0) and not dbg["xq"].cpu().numpy().any()
+    finally:
+        L.close()
+    lw = synth.layer_weights(3, 0, E, H, I)
+    lw["w13_codes"][:] = 0
+    L = GpuLayer(3, 0, E, H, I, k=2, weights=lw)
+    try:
+        x = synth.hidden_states(3, 1, 1, H)
+        ids, w, counts, y, dbg = _run(L, x)
+        assert not (u16(y) & 0x7FFF).any()
+    finally:
+        L.close()
+
+
+def test_gpu_bad_ids_are_reported_and_skipped():
+    E, H, I = 8, 128, 64
+    L = GpuLayer(4, 0, E, H, I, k=2, fill="host")
+    try:
+        x = synth.hidden_states(4, 0, 1, H)
+        xd = to_dev_u16(x)
+        ids = torch.tensor([[1, 99]], dtype=torch.int32, device="cuda")
+        w = torch.tensor([[0.75, 0.25]], dtype=torch.float32, device="cuda")
+        y, _ = L.forward(xd, 1, ids, w, debug=False)
+        assert moe.moe_device_error(L.handle) == moe.MOE_ERR_DEVICE
+        assert moe.moe_device_error(L.handle) == moe.MOE_OK      # cleared
+        # the valid slot and the shared expert still count
+        ref = OM.moe_forward(x, np.array([[1]], np.int32), np.array([[0.75]], np.float32),
+                             L.host, E, I, 1)
+        yg, yr = OF.bf16_to_f64(u16(y)), OF.bf16_to_f64(ref["y"])
+        assert np.linalg.norm(yg - yr) <= 2e-3 * np.linalg.norm(yr)
+    finally:
+        L.close()
+
+
+def test_gpu_token_count_limits():
+    L = GpuLayer(0, 0, 8, 128, 64, k=2, fill="host", max_tokens=4)
+    try:
+        x = to_dev_u16(np.zeros((8, 128), np.uint16))
+        ids = torch.zeros((8, 2), dtype=torch.int32, device="cuda")
+        w = torch.zeros((8, 2), dtype=torch.float32, device="cuda")
+        y = torch.empty((8, 128), dtype=torch.int16, device="cuda")
+        for T in (0, 5):
+            with pytest.raises(moe.MoEError) as ei:
+                moe.moe_forward(L.handle, x, T, ids, w, y)
+            assert ei.value.code == moe.MOE_ERR_ARG
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_route(L.handle, x.data_ptr() + 2, 1, ids, w)
+        assert ei.value.code == moe.MOE_ERR_ALIGN
+    finally:
+        L.close()
+
+
+def test_gpu_residual_rmsnorm_matches_oracle():
+    T, H = 3, 2560
+    r = synth.hidden_states(7, 0, T, H)
+    y = synth.hidden_states(7, 1, T, H)
+    rd, yd = to_dev_u16(r), to_dev_u16(y)
+    xn = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    moe.moe_residual_rmsnorm(rd, yd, xn, T, H, 1e-6)
+    rr, rx = OM.residual_rmsnorm(r, y, 1e-6)
+    assert np.array_equal(u16(rd), rr)
+    assert np.array_equal(u16(xn), rx)
