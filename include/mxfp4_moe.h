@@ -70,24 +70,41 @@ typedef struct {
   int32_t n_shared;   /* shared experts, 0..2, added with weight 1         */
 } moe_config;
 
-/* All device pointers, borrowed: they must stay valid while the handle is
- * used.  Expert arrays hold the routed experts 0..E-1 followed by the shared
+/* MXFP4 expert weights in the plain (canonical) layout, device pointers.
+ * Expert arrays hold the routed experts 0..E-1 followed by the shared
  * experts E..E+n_shared-1, each expert contiguous:
  *   w13_codes  [E+S][2I][H/2]  rows 0..I-1 gate, rows I..2I-1 up (uint8)
  *   w13_scales [E+S][2I][H/32] E8M0 exponents (uint8)
  *   w2_codes   [E+S][H][I/2]   down projection
  *   w2_scales  [E+S][H][I/32]
- *   router_w   [E][H]          bfloat16 bit patterns (uint16)
- *   router_bias[E]             float32, or NULL for no bias
- * E8M0 exponent 255 (NaN) is not supported. */
+ * E8M0 exponent 255 (NaN) is not supported.  This is the input of
+ * moe_pack_weights; the layer itself reads the packed layout below. */
 typedef struct {
-  const uint16_t* router_w;
-  const float* router_bias;
   const uint8_t* w13_codes;
   const uint8_t* w13_scales;
   const uint8_t* w2_codes;
   const uint8_t* w2_scales;
+} moe_mxfp4_weights;
+
+/* Weights of one layer as the kernels read them (device pointers, borrowed:
+ * they must stay valid while the handle is used):
+ *   router_w   [E][H]  bfloat16 bit patterns (uint16)
+ *   router_bias[E]     float32, or NULL for no bias
+ *   w13        [E+S][I/8][MOE_W13_TILE_BYTES(H)]  packed gate/up tiles
+ *   w2         [E+S][H/16][MOE_W2_TILE_BYTES(I)]  packed down tiles
+ * The packed arrays hold exactly the bytes of the canonical layout,
+ * reordered by moe_pack_weights so that every 16-row tile of every 32-element
+ * block is contiguous in the order the tensor-core fragments are loaded
+ * (see moe_pack_weights). */
+typedef struct {
+  const uint16_t* router_w;
+  const float* router_bias;
+  const uint8_t* w13;
+  const uint8_t* w2;
 } moe_weights;
+
+#define MOE_W13_TILE_BYTES(H) (272 * ((H) / 32))  /* 8 gate + 8 up rows */
+#define MOE_W2_TILE_BYTES(I) (272 * ((I) / 32))   /* 16 down rows */
 
 /* Optional debug outputs of moe_forward (device pointers, each may be NULL):
  *   xq [T][H] FP8 codes of x, xs [T] their scales,
@@ -153,6 +170,22 @@ int moe_destroy(moe_handle h);
 
 /* Static text for a return code. */
 const char* moe_strerror(int code);
+
+/* Reorder canonical MXFP4 expert weights into the packed layout the
+ * kernels read, for experts expert0 .. expert0+n_experts-1 (shared experts
+ * included by index).  No value changes: every byte of the input appears once
+ * in the output.  Layout of one gate/up tile (features j0..j0+7, j0 = 8c):
+ * for each 32-element block b: 256 code bytes, for lane L = 4g+t (g 0..7,
+ * t 0..3) the 4 bytes 16b+4t.. of gate row j0+g then those of up row j0+g;
+ * then for each block 16 scale bytes (gate row j0+g, up row j0+g) for
+ * g = 0..7.  A down tile (rows n0..n0+15, n0 = 16p) is the same with row
+ * n0+g in place of the gate row and n0+g+8 in place of the up row.  Output
+ * buffers are caller-allocated ([E+S][I/8][MOE_W13_TILE_BYTES(H)] and
+ * [E+S][H/16][MOE_W2_TILE_BYTES(I)]); the call only enqueues a kernel.
+ * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_ALIGN. */
+int moe_pack_weights(const moe_config* cfg, const moe_mxfp4_weights* src, int expert0,
+                     int n_experts, uint8_t* w13_packed, uint8_t* w2_packed,
+                     cudaStream_t stream);
 
 /* Per-row FP8 E4M3 quantisation, the activation step of the W4A8 recipe
  * (tanhow.com retelling, "为什么 DGX Spark 上的 MoE 解码是内存受限的？";

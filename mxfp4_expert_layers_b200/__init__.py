@@ -27,7 +27,7 @@ MOE_GEMV_MAX_TOKENS = 4
 
 EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
-           "moe_profile_begin", "moe_profile_end")
+           "moe_profile_begin", "moe_profile_end", "moe_pack_weights")
 MOE_PROFILE_KERNELS = 4
 KERNEL_NAMES = ("route", "gateup_swiglu", "down_combine", "reserved")
 
@@ -44,10 +44,22 @@ class moe_config(ctypes.Structure):
                 ("n_shared", ctypes.c_int32)]
 
 
+class moe_mxfp4_weights(ctypes.Structure):
+    _fields_ = [("w13_codes", ctypes.c_void_p), ("w13_scales", ctypes.c_void_p),
+                ("w2_codes", ctypes.c_void_p), ("w2_scales", ctypes.c_void_p)]
+
+
 class moe_weights(ctypes.Structure):
     _fields_ = [("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
-                ("w13_codes", ctypes.c_void_p), ("w13_scales", ctypes.c_void_p),
-                ("w2_codes", ctypes.c_void_p), ("w2_scales", ctypes.c_void_p)]
+                ("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p)]
+
+
+def w13_tile_bytes(hidden: int) -> int:
+    return 272 * (hidden // 32)
+
+
+def w2_tile_bytes(inter: int) -> int:
+    return 272 * (inter // 32)
 
 
 class moe_debug(ctypes.Structure):
@@ -74,6 +86,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_destroy.argtypes = [p]
     L.moe_strerror.argtypes = [i]
     L.moe_strerror.restype = ctypes.c_char_p
+    L.moe_pack_weights.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_mxfp4_weights), i, i,
+                                    p, p, p]
     L.moe_profile_begin.argtypes = [p, i]
     L.moe_profile_end.argtypes = [p, p, p]
     L.moe_quantize_fp8.argtypes = [p, i, i, p, p, p]
@@ -114,10 +128,22 @@ def strerror(code: int) -> str:
 moe_strerror = strerror
 
 
+def moe_pack_weights(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
+                     src: dict, expert0: int, count: int, w13_packed, w2_packed, stream=None) -> None:
+    """Reorder canonical MXFP4 weights (``src``: w13_codes, w13_scales,
+    w2_codes, w2_scales tensors) into the packed layout, experts
+    ``expert0 .. expert0+count-1``."""
+    cfg = moe_config(hidden, inter, n_experts, top_k, n_shared)
+    w = moe_mxfp4_weights(*[_ptr(src.get(f)) for f, _ in moe_mxfp4_weights._fields_])
+    _check(load().moe_pack_weights(ctypes.byref(cfg), ctypes.byref(w), expert0, count, _ptr(w13_packed),
+                                   _ptr(w2_packed), _stream(stream)), "moe_pack_weights")
+
+
 def moe_create(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
                weights: dict, max_tokens: int) -> int:
     """Returns an opaque handle.  ``weights`` maps the moe_weights field names
-    to CUDA tensors (``router_bias`` may be None)."""
+    (router_w, router_bias, w13, w2 -- packed) to CUDA tensors
+    (``router_bias`` may be None)."""
     cfg = moe_config(hidden, inter, n_experts, top_k, n_shared)
     w = moe_weights(*[_ptr(weights.get(f)) for f, _ in moe_weights._fields_])
     h = ctypes.c_void_p()

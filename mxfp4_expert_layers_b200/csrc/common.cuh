@@ -168,10 +168,63 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only, not L1), and the
+// mbarrier arrival that fires when all of this thread's earlier cp.async
+// copies have landed (the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// L2 prefetch of a global range (16-byte multiple), no shared memory involved.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ------------------------------------------------ programmatic dependent launch --
+// griddepcontrol.wait: block until the grids this one depends on have
+// completed and their memory is visible.  launch_dependents: allow the next
+// kernel of the stream to start launching (its pre-wait code overlaps ours).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------ tensor cores --
+// D = A * B + C, m16n8k16, A/B f16, C/D f32 (mma.sync).  Fragments:
+//   a0 = A[g][2t..2t+1], a1 = A[g+8][2t..], a2 = A[g][2t+8..], a3 = A[g+8][2t+8..]
+//   b0 = B[2t..2t+1][g], b1 = B[2t+8..2t+9][g]
+//   d0 = D[g][2t], d1 = D[g][2t+1], d2 = D[g+8][2t], d3 = D[g+8][2t+1]
+// with g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1, const float (&c)[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+        "f"(c[2]), "f"(c[3]));
+}
+
+// byte `i` of a word of E2M1 codes -> f16x2 bits (low nibble in the low half)
+__device__ __forceinline__ uint32_t e2m1x2_bits(uint32_t word, int i) {
+  __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>((word >> (8 * i)) & 0xFFu),
+                                             __NV_E2M1);
+  return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+}
+
+// two E4M3 bytes (low byte first) -> f16x2 bits
+__device__ __forceinline__ uint32_t e4m3x2_bits(uint32_t two) {
+  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+}
+
 // ------------------------------------------------------------- dispatch --
-// Distinct experts of a small call (T <= kMaxTokGemv), in order of first
-// appearance over (token, slot), shared experts last.  Every kernel of the
-// GEMV path rebuilds the same list from the ids.
+// Distinct experts of a small call (T <= kMaxTokGemv): the shared experts
+// first, then the routed ones in order of first appearance over (token,
+// slot).  Every kernel of the GEMV path rebuilds the same list from the ids.
 struct Distinct {
   int n;                                  // number of distinct experts
   int expert[kMaxDistinct];               // expert index (shared: E + s)

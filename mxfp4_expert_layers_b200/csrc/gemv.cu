@@ -1,25 +1,35 @@
 // Split-K MXFP4 GEMV path of the MoE layer for 1..4 tokens (decode and
 // speculative verify: "三项优化是什么？" item 3 of the tanhow.com retelling --
-// 4 verified tokens touch up to 32 experts).
+// verifying 4 tokens touches up to 32 experts).
 //
-// Two kernels, each streaming its weight slabs global -> shared with 1-D
-// bulk copies (TMA, no multicast) completing on an mbarrier:
+// Weights are read in the packed tile layout (moe_pack_weights): for every
+// 16-row tile and 32-element block, lane L = 4g+t of a warp owns 8 contiguous
+// bytes -- word t of tile rows g and g+8 -- so a warp's load of a block is
+// 256 contiguous bytes and lands directly in its tensor-core fragments.
 //
-//  gateup_swiglu: CTA = (distinct expert u, 16 features j).  Copies the 16
-//    gate rows and 16 up rows it needs (40 KB at H = 2560) while it
-//    quantises x to FP8 E4M3 (per-token amax / 448), then computes
-//    g = xs * sum_b 2^(E_b-127) * S_b with S_b the 32-term block sum in
-//    float32 (exact: every product of an E2M1 and an E4M3 value has at most
-//    6 significant bits) and the cross-block sum in float64 (exact for the
-//    layer's value range), so g and u equal the oracle's bit for bit.
-//    h = silu(g) * u in float64, stored as float32.  The last CTA of each
-//    expert (atomic counter, no waiting) re-quantises that expert's h to
-//    FP8 with its amax / 448.
-//  down_combine: CTA = 8 output rows.  Streams the 8-row slab of every
-//    distinct expert through a ring of stages and accumulates
-//    sum_u w_u * sh_u * sum_b 2^(E-127) * S_b in float64 per (row, token);
-//    the expert reduction stays inside the CTA (no atomics), then one
-//    rounding to bfloat16.
+// Arithmetic per block: the E2M1 codes are placed in E4M3 bytes (3 magnitude
+// bits at bits 4..2, sign at bit 7), which represents every E2M1 value times
+// 2^-6 exactly, subnormal 0.5 included; activations are FP8 E4M3 already.  One
+// mma.sync m16n8k32 (e4m3 x e4m3 -> f32) gives the 32-element block sums of
+// 16 rows x 8 token columns; those sums are exact in f32 (at most 6
+// significant bits per product).  Each block sum is scaled by 2^(E-127+6)
+// and accumulated in float64, so g and u equal the oracle's bit for bit.
+//
+//  gateup_swiglu (one CTA per SM, 16 warps): the distinct experts of the
+//    call (shared first) are cut into chunks of 8 features (one tile: 8 gate
+//    + 8 up rows); chunk c belongs to CTA c mod G.  The 16 warps split each
+//    chunk's blocks; loads of the next chunk are in flight while the current
+//    one is computed.  Partial sums go to shared memory with float64 atomic
+//    adds (exact, so the order does not matter); one barrier at the end, then
+//    the SwiGLU of every feature: h = silu(g) * u in float64, stored as
+//    float32, and a per-(expert, token) amax kept by atomicMax.  x is
+//    quantised to FP8 (amax / 448) before the dependency wait.
+//  down_combine (one 16-row tile per CTA): before its wait it rebuilds the
+//    expert list and loads the tile's fragments of every expert's down weights
+//    into registers (prefetched into L2 by the gate/up CTAs); after the wait
+//    it re-quantises h to FP8 with amax / 448 and sums
+//    w * sh * 2^(E-127+6) * S_b in float64 over blocks and experts inside the
+//    CTA, then rounds once to bfloat16.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -27,389 +37,529 @@ namespace moe {
 
 namespace {
 
-constexpr int kJT = 16;          // features per gate/up CTA
-constexpr int kGUThreads = 256;  // 8 warps = 16 half-warps, one feature each
-constexpr int kNT = 8;           // output rows per down CTA
-constexpr int kStages = 12;      // expert slabs in flight per down CTA
+constexpr int kGUThreads = 512;   // 16 warps
+constexpr int kGUWarps = kGUThreads / 32;
+constexpr int kDNThreads = 256;   // 8 warps
+constexpr int kDNWarps = kDNThreads / 32;
+constexpr int kChunkF = 8;        // features per chunk (16 rows with gate + up)
+constexpr int kDNBatch = 28;      // (expert, block) pairs per warp held in registers
 
 __host__ __device__ constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ constexpr size_t tile_bytes(int K) { return 272u * static_cast<size_t>(K / 32); }
 
 // ---------------------------------------------------------------- dispatch --
-__device__ void build_distinct(const int32_t* ids, const float* w, int T, int k, int E,
-                               int n_shared, Distinct& d, double (*wsum)[kMaxTokGemv],
-                               int* err, bool report) {
-  d.n = 0;
-  for (int t = 0; t < T; ++t) {
-    for (int i = 0; i < k; ++i) {
-      const int e = ids[t * k + i];
-      if (e < 0 || e >= E) {
-        if (report) atomicOr(err, kErrBadId);
-        continue;
-      }
-      int j = 0;
-      while (j < d.n && d.expert[j] != e) ++j;
-      if (j == d.n) {
-        d.expert[j] = e;
-        d.mask[j] = 0;
-        for (int tt = 0; tt < kMaxTokGemv; ++tt) wsum[j][tt] = 0.0;
-        d.n++;
-      }
-      d.mask[j] |= static_cast<uint8_t>(1u << t);
-      if (w) wsum[j][t] += static_cast<double>(w[t * k + i]);
-    }
+// The distinct experts of the call, built by one warp: shared experts first,
+// then routed experts in order of first appearance over (token, slot).  With
+// w given, wsum gets the summed routing weight per (expert, token).
+__device__ void build_distinct_warp(const int32_t* ids, const float* w, int T, int k, int E,
+                                    int n_shared, Distinct& d, double (*wsum)[kMaxTokGemv],
+                                    int* err, bool report) {
+  const int lane = threadIdx.x & 31;
+  const int n = T * k;  // <= 32
+  for (int i = lane; i < kMaxDistinct; i += 32) {
+    d.mask[i] = 0;
+    for (int t = 0; t < kMaxTokGemv; ++t) wsum[i][t] = 0.0;
   }
-  for (int s = 0; s < n_shared; ++s) {
-    const int j = d.n++;
-    d.expert[j] = E + s;
-    d.mask[j] = static_cast<uint8_t>((1u << T) - 1);
-    for (int tt = 0; tt < kMaxTokGemv; ++tt) wsum[j][tt] = 1.0;
+  __syncwarp();
+  const int e = lane < n ? ids[lane] : -1;
+  const bool valid = lane < n && e >= 0 && e < E;
+  if (lane < n && !valid && report) atomicOr(err, kErrBadId);
+  int first = lane;  // first lane holding the same expert
+  for (int j = 0; j < n; ++j) {
+    const int ej = __shfl_sync(0xffffffffu, e, j);
+    if (j < first && ej == e) first = j;
   }
+  const unsigned lead = __ballot_sync(0xffffffffu, valid && first == lane);
+  const int pos = __popc(lead & ((1u << lane) - 1u));
+  if (valid && first == lane) d.expert[n_shared + pos] = e;
+  const int my_u = n_shared + __shfl_sync(0xffffffffu, pos, first);
+  if (lane < n_shared) {
+    d.expert[lane] = E + lane;
+    d.mask[lane] = static_cast<uint8_t>((1u << T) - 1);
+    for (int t = 0; t < kMaxTokGemv; ++t) wsum[lane][t] = 1.0;
+  }
+  __syncwarp();
+  if (valid) {
+    const int t = lane / k;
+    atomicOr(reinterpret_cast<unsigned*>(&d.mask[0]) + (my_u >> 2), 1u << (8 * (my_u & 3) + t));
+    if (w) atomicAdd(&wsum[my_u][t], static_cast<double>(w[lane]));
+  }
+  if (lane == 0) d.n = n_shared + __popc(lead);
+  __syncwarp();
 }
 
-// Exact block sum of 32 products: E2M1 codes (16 bytes) x half activations
-// (32 halves, element order matching the codes: element 2i = low nibble of
-// byte i).
-__device__ __forceinline__ float block_dot(const uint4 c, const uint4* act) {
-  float s = 0.f;
-  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 av = act[q];
-    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 wf = __half22float2(e2m1x2_to_half2(cw[q] >> (8 * i)));
-      const float2 af = __half22float2(*reinterpret_cast<const __half2*>(&aw[i]));
-      s = fmaf(wf.x, af.x, s);
-      s = fmaf(wf.y, af.y, s);
-    }
-  }
-  return s;
+// 8 E2M1 codes (one word) -> E4M3 bytes holding value * 2^-6: the codes of
+// the high nibbles (elements 1, 3, 5, 7) and of the low nibbles (0, 2, 4, 6)
+__device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) { return (w & 0x80808080u) | ((w & 0x70707070u) >> 2); }
+__device__ __forceinline__ uint32_t e4m3_lo(uint32_t w) { return e4m3_hi(w << 4); }
+
+// D = A * B (+ C), m16n8k32, A/B e4m3, C/D f32 (mma.sync).  Fragments:
+//   a0 = A[g][4t..4t+3], a1 = A[g+8][4t..], a2 = A[g][16+4t..], a3 = A[g+8][16+4t..]
+//   b0 = B[4t..4t+3][g], b1 = B[16+4t..16+4t+3][g]
+//   d0 = D[g][2t], d1 = D[g][2t+1], d2 = D[g+8][2t], d3 = D[g+8][2t+1]
+__device__ __forceinline__ void mma_fp8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// Position of element k (0..31) of a block inside its permuted activation
+// bytes: group k/8 holds [k0 k2 k4 k6 k1 k3 k5 k7] of that group.
+__device__ __forceinline__ int perm_pos(int k) {
+  const int kk = k & 7;
+  return (k & ~7) + ((kk & 1) ? 4 + (kk >> 1) : (kk >> 1));
 }
 
 // ------------------------------------------------------------ gate / up ---
-struct GUSmem {
-  __host__ __device__ static size_t codes(int H) { return align_up(static_cast<size_t>(kJT) * H / 2, 128); }
-  __host__ __device__ static size_t scales(int H) { return align_up(static_cast<size_t>(kJT) * H / 32, 128); }
-  __host__ __device__ static size_t act(int H, int T) { return align_up(static_cast<size_t>(T) * H * 2, 128); }
-  __host__ __device__ static size_t total(int H, int T) { return 2 * codes(H) + 2 * scales(H) + act(H, T); }
+struct GU {
+  __host__ __device__ static size_t act(int H, int T) { return align_up(static_cast<size_t>(T) * H, 128); }
+  __host__ __device__ static size_t red(int T, int nmax) {
+    return align_up(static_cast<size_t>(nmax) * 16 * T * sizeof(double), 128);
+  }
+  __host__ __device__ static size_t total(int H, int T, int nmax) { return act(H, T) + red(T, nmax); }
 };
 
+template <int NBW>  // blocks per warp per chunk: ceil((H/32) / 16)
 __global__ void __launch_bounds__(kGUThreads)
 gateup_swiglu_kernel(GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Distinct dist;
   __shared__ double wsum[kMaxDistinct][kMaxTokGemv];
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ float red[kGUThreads / 32];
+  __shared__ float red_f[kGUWarps];
   __shared__ float xs[kMaxTokGemv];
-  __shared__ int s_flag;
+  __shared__ int s_ids[kMaxTokGemv * MOE_MAX_TOPK];
+  __shared__ unsigned amax_l[kMaxDistinct][kMaxTokGemv];
 
   const int H = a.H, I = a.I, T = a.T;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u = blockIdx.y;
-  const int j0 = blockIdx.x * kJT;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int cpe = I / kChunkF, nb = H / 32;
+  uint8_t* s_act = smem;                                            // [T][H] permuted E4M3
+  double* s_red = reinterpret_cast<double*>(smem + GU::act(H, T));  // [chunk][16][T]
 
-  if (tid == 0)
-    build_distinct(a.ids, nullptr, T, a.k, a.E, a.n_shared, dist, wsum, a.err,
-                   blockIdx.x == 0 && blockIdx.y == 0);
-  __syncthreads();
-  if (u >= dist.n) return;
-  const int e = dist.expert[u];
-  const unsigned mask = dist.mask[u];
+  for (int i = tid; i < kMaxDistinct * kMaxTokGemv; i += kGUThreads) (&amax_l[0][0])[i] = 0u;
+  for (int i = tid; i < a.gu_nmax * 16 * T; i += kGUThreads) s_red[i] = 0.0;
 
-  uint8_t* s_codes = smem;                               // [2][kJT][H/2]
-  uint8_t* s_scl = smem + 2 * GUSmem::codes(H);          // [2][kJT][H/32]
-  __half* s_act = reinterpret_cast<__half*>(s_scl + 2 * GUSmem::scales(H));  // [T][H]
-
-  // ---- issue the weight copies (one thread), then quantise x meanwhile
-  const size_t rowb = H / 2, rows_scl = H / 32;
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-    const uint32_t cbytes = kJT * rowb, sbytes = kJT * rows_scl;
-    mbar_expect_tx(&bar, 2 * cbytes + 2 * sbytes);
-    const uint8_t* cbase = a.w13_codes + static_cast<size_t>(e) * 2 * I * rowb;
-    const uint8_t* sbase = a.w13_scales + static_cast<size_t>(e) * 2 * I * rows_scl;
-    bulk_g2s(s_codes, cbase + j0 * rowb, cbytes, &bar);
-    bulk_g2s(s_codes + GUSmem::codes(H), cbase + (I + j0) * rowb, cbytes, &bar);
-    bulk_g2s(s_scl, sbase + j0 * rows_scl, sbytes, &bar);
-    bulk_g2s(s_scl + GUSmem::scales(H), sbase + (I + j0) * rows_scl, sbytes, &bar);
-  }
-
-  const bool dbg_writer = (blockIdx.x == 0 && u == 0);
+  // ---- before the dependency wait: quantise x (an input of the call)
+  const bool dbg_writer = cta == 0;
   for (int t = 0; t < T; ++t) {
-    const uint16_t* xr = a.x + static_cast<size_t>(t) * H;
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * H);
+    const int units = H / 8;
+    uint4 v[2];
     float m = 0.f;
-    for (int i = tid; i < H; i += kGUThreads) m = fmaxf(m, fabsf(bf16_bits_to_f32(xr[i])));
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + r * kGUThreads;
+      v[r] = i < units ? __ldcg(xr + i) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t wv[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[j] << 16)), fabsf(__uint_as_float(wv[j] & 0xFFFF0000u))));
+    }
+    for (int i = tid + 2 * kGUThreads; i < units; i += kGUThreads) {  // wide rows
+      const uint4 u = __ldcg(xr + i);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+      for (int j = 0; j < 4; ++j)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(wv[j] << 16)), fabsf(__uint_as_float(wv[j] & 0xFFFF0000u))));
+    }
     m = warp_max_f32(m);
-    if (lane == 0) red[warp] = m;
+    if (lane == 0) red_f[warp] = m;
     __syncthreads();
     if (tid == 0) {
       float amax = 0.f;
-      for (int i = 0; i < kGUThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+      for (int i = 0; i < kGUWarps; ++i) amax = fmaxf(amax, red_f[i]);
       xs[t] = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
       if (dbg_writer && a.dbg.xs) a.dbg.xs[t] = xs[t];
     }
     __syncthreads();
     const float s = xs[t];
-    for (int i = tid; i < H; i += kGUThreads) {
-      const uint8_t q = f32_to_e4m3(__fdiv_rn(bf16_bits_to_f32(xr[i]), s));
-      s_act[static_cast<size_t>(t) * H + i] = e4m3_to_half(q);
-      if (dbg_writer && a.dbg.xq) a.dbg.xq[static_cast<size_t>(t) * H + i] = q;
-    }
-  }
-  __syncthreads();
-
-  if (!mbar_wait_bounded(&bar, 0, a.err)) {
-    // give up without computing; let the copies land (again bounded) before
-    // the CTA's shared memory is released
-    mbar_wait_bounded(&bar, 0, nullptr);
-    return;
-  }
-
-  // ---- dot products: half-warp hw of warp w owns feature jj = 2w + hw
-  const int hw = lane >> 4, sl = lane & 15;
-  const int jj = 2 * warp + hw;
-  const int nb = H / 32;
-  double acc_g[kMaxTokGemv], acc_u[kMaxTokGemv];
+    // quantise from the registers loaded above (8 values per 16-byte unit)
 #pragma unroll
-  for (int t = 0; t < kMaxTokGemv; ++t) acc_g[t] = acc_u[t] = 0.0;
-
-  const uint8_t* cg = s_codes + static_cast<size_t>(jj) * rowb;
-  const uint8_t* cu = s_codes + GUSmem::codes(H) + static_cast<size_t>(jj) * rowb;
-  const uint8_t* sg = s_scl + static_cast<size_t>(jj) * rows_scl;
-  const uint8_t* su = s_scl + GUSmem::scales(H) + static_cast<size_t>(jj) * rows_scl;
-  for (int b = sl; b < nb; b += 16) {
-    const uint4 wg = *reinterpret_cast<const uint4*>(cg + b * 16);
-    const uint4 wu = *reinterpret_cast<const uint4*>(cu + b * 16);
-    const double fg = e8m0_to_f64(sg[b]);
-    const double fu = e8m0_to_f64(su[b]);
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + r * kGUThreads;
+      if (i < units) {
+        const uint32_t wv[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+        uint8_t* dst = s_act + static_cast<size_t>(t) * H + 8 * (i & ~3);
 #pragma unroll
-    for (int t = 0; t < kMaxTokGemv; ++t) {
-      if (t < T && (mask >> t & 1)) {
-        const uint4* act = reinterpret_cast<const uint4*>(s_act + static_cast<size_t>(t) * H + b * 32);
-        acc_g[t] = fma(static_cast<double>(block_dot(wg, act)), fg, acc_g[t]);
-        acc_u[t] = fma(static_cast<double>(block_dot(wu, act)), fu, acc_u[t]);
-      }
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < kMaxTokGemv; ++t) {
-    if (t < T && (mask >> t & 1)) {
-      const double G = warp_sum_f64(acc_g[t], 16);
-      const double U = warp_sum_f64(acc_u[t], 16);
-      if (sl == 0) {
-        const double g = static_cast<double>(xs[t]) * G;
-        const double uu = static_cast<double>(xs[t]) * U;
-        const double hv = g / (1.0 + exp(-g)) * uu;
-        a.h[(static_cast<size_t>(u) * kMaxTokGemv + t) * I + j0 + jj] = static_cast<float>(hv);
-      }
-    }
-  }
-
-  // ---- last CTA of this expert: FP8 re-quantisation of h per token
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int old = atomicAdd(&a.expert_counter[u], 1);
-    s_flag = (old == static_cast<int>(gridDim.x) - 1);
-  }
-  __syncthreads();
-  if (!s_flag) return;
-  __threadfence();
-  for (int t = 0; t < T; ++t) {
-    if (!(mask >> t & 1)) continue;
-    const float* hr = a.h + (static_cast<size_t>(u) * kMaxTokGemv + t) * I;
-    float m = 0.f;
-    for (int j = tid; j < I; j += kGUThreads) m = fmaxf(m, fabsf(__ldcg(hr + j)));
-    m = warp_max_f32(m);
-    if (lane == 0) red[warp] = m;
-    __syncthreads();
-    if (tid == 0) {
-      float amax = 0.f;
-      for (int i = 0; i < kGUThreads / 32; ++i) amax = fmaxf(amax, red[i]);
-      xs[0] = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);  // reuse as s_h
-      a.sh[static_cast<size_t>(u) * kMaxTokGemv + t] = xs[0];
-    }
-    __syncthreads();
-    const float shv = xs[0];
-    uint8_t* qr = a.qh + (static_cast<size_t>(u) * kMaxTokGemv + t) * I;
-    // debug slots of this token that route to expert e
-    const int S = a.k + a.n_shared;
-    for (int j = tid; j < I; j += kGUThreads) {
-      const float hv = __ldcg(hr + j);
-      const uint8_t q = f32_to_e4m3(__fdiv_rn(hv, shv));
-      qr[j] = q;
-      if (a.dbg.qh || a.dbg.h) {
-        for (int sidx = 0; sidx < S; ++sidx) {
-          const int es = sidx < a.k ? a.ids[t * a.k + sidx] : a.E + (sidx - a.k);
-          if (es != e) continue;
-          const size_t o = (static_cast<size_t>(t) * S + sidx) * I + j;
-          if (a.dbg.qh) a.dbg.qh[o] = q;
-          if (a.dbg.h) a.dbg.h[o] = hv;
+        for (int jj = 0; jj < 8; ++jj) {
+          const int k = 8 * i + jj;
+          const float xv = __uint_as_float(jj & 1 ? (wv[jj >> 1] & 0xFFFF0000u) : (wv[jj >> 1] << 16));
+          const uint8_t q = f32_to_e4m3(__fdiv_rn(xv, s));
+          dst[perm_pos(k & 31)] = q;
+          if (dbg_writer && a.dbg.xq) a.dbg.xq[static_cast<size_t>(t) * H + k] = q;
         }
       }
     }
-    if (tid == 0 && a.dbg.sh) {
-      for (int sidx = 0; sidx < S; ++sidx) {
-        const int es = sidx < a.k ? a.ids[t * a.k + sidx] : a.E + (sidx - a.k);
-        if (es == e) a.dbg.sh[static_cast<size_t>(t) * S + sidx] = shv;
+    for (int i = tid + 2 * kGUThreads; i < units; i += kGUThreads) {  // wide rows
+      const uint4 u4 = __ldcg(xr + i);
+      const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
+      uint8_t* dst = s_act + static_cast<size_t>(t) * H + 8 * (i & ~3);
+      for (int jj = 0; jj < 8; ++jj) {
+        const int k = 8 * i + jj;
+        const float xv = __uint_as_float(jj & 1 ? (wv[jj >> 1] & 0xFFFF0000u) : (wv[jj >> 1] << 16));
+        const uint8_t q = f32_to_e4m3(__fdiv_rn(xv, s));
+        dst[perm_pos(k & 31)] = q;
+        if (dbg_writer && a.dbg.xq) a.dbg.xq[static_cast<size_t>(t) * H + k] = q;
       }
     }
-    __syncthreads();
   }
-  if (tid == 0) a.expert_counter[u] = 0;
+
+  // ---- routing of this call (written by the router kernel)
+  pdl_wait();
+  if (warp == 0) {
+    if (lane < T * a.k) s_ids[lane] = __ldcg(a.ids + lane);
+    __syncwarp();
+    build_distinct_warp(s_ids, nullptr, T, a.k, a.E, a.n_shared, dist, wsum, a.err, dbg_writer);
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  const int nchunks = dist.n * cpe;
+  const int nmine = cta < nchunks ? (nchunks - 1 - cta) / G + 1 : 0;
+  // L2 prefetch of the down weights this call needs: CTA b takes a slice of
+  // every expert's packed down weights
+  if (warp == 1 && a.prefetch_down) {
+    const size_t eb = static_cast<size_t>(H / 16) * tile_bytes(I);
+    const size_t s0 = (eb * cta / G) & ~static_cast<size_t>(15);
+    const size_t s1 = (eb * (cta + 1) / G) & ~static_cast<size_t>(15);
+    if (s1 > s0)
+      for (int u = lane; u < dist.n; u += 32)
+        prefetch_l2(a.w2 + static_cast<size_t>(dist.expert[u]) * eb + s0, static_cast<uint32_t>(s1 - s0));
+  }
+
+  const int g = lane >> 2, t = lane & 3;
+  const int bw0 = warp * NBW;
+  const size_t tb = tile_bytes(H);
+  // fragments of one chunk: word pairs and scale pairs of this lane's blocks
+  uint2 cw[2][NBW];
+  uint32_t sc[2][NBW];
+  auto load = [&](int j, int buf) {
+    const int c = cta + G * j;
+    const uint8_t* base = a.w13 + (static_cast<size_t>(dist.expert[c / cpe]) * cpe + c % cpe) * tb;
+#pragma unroll
+    for (int i = 0; i < NBW; ++i) {
+      const int b = bw0 + i;
+      if (b < nb) {
+        cw[buf][i] = __ldcs(reinterpret_cast<const uint2*>(base + 256 * b) + lane);
+        sc[buf][i] = __ldcs(reinterpret_cast<const uint16_t*>(base + 256 * nb + 16 * b) + g);
+      }
+    }
+  };
+  auto compute = [&](int j, int buf) {
+    const int c = cta + G * j;
+    const int u = c / cpe;
+    const unsigned mask = dist.mask[u];
+    const bool tok = g < T && (mask >> g & 1);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int i = 0; i < NBW; ++i) {
+      const int b = bw0 + i;
+      if (b < nb) {
+        const uint32_t wa = cw[buf][i].x, wb = cw[buf][i].y;
+        const uint32_t af[4] = {e4m3_lo(wa), e4m3_lo(wb), e4m3_hi(wa), e4m3_hi(wb)};
+        uint2 q = make_uint2(0u, 0u);
+        if (tok) q = *reinterpret_cast<const uint2*>(s_act + static_cast<size_t>(g) * H + 32 * b + 8 * t);
+        float d[4];
+        mma_fp8(d, af, q.x, q.y);
+        if (2 * t < T) {
+          const double fa = e8m0_to_f64((sc[buf][i] & 0xFFu) + 6), fb = e8m0_to_f64((sc[buf][i] >> 8) + 6);
+          acc[0] = fma(static_cast<double>(d[0]), fa, acc[0]);
+          acc[2] = fma(static_cast<double>(d[2]), fb, acc[2]);
+          if (2 * t + 1 < T) {
+            acc[1] = fma(static_cast<double>(d[1]), fa, acc[1]);
+            acc[3] = fma(static_cast<double>(d[3]), fb, acc[3]);
+          }
+        }
+      }
+    }
+    // exact partial sums: order-free float64 atomics
+    double* red = s_red + static_cast<size_t>(j) * 16 * T;
+    if (2 * t < T && bw0 < nb) {
+      atomicAdd(&red[g * T + 2 * t], acc[0]);
+      atomicAdd(&red[(g + 8) * T + 2 * t], acc[2]);
+      if (2 * t + 1 < T) {
+        atomicAdd(&red[g * T + 2 * t + 1], acc[1]);
+        atomicAdd(&red[(g + 8) * T + 2 * t + 1], acc[3]);
+      }
+    }
+  };
+  if (nmine > 0) load(0, 0);
+  for (int j = 0; j < nmine; j += 2) {
+    if (j + 1 < nmine) load(j + 1, 1);
+    compute(j, 0);
+    if (j + 2 < nmine) load(j + 2, 0);
+    if (j + 1 < nmine) compute(j + 1, 1);
+  }
+  __syncthreads();
+  // SwiGLU of every feature of every chunk of this CTA
+  for (int p = tid; p < nmine * kChunkF * T; p += kGUThreads) {
+    const int j = p / (kChunkF * T), r = p % (kChunkF * T), f = r / T, tt = r % T;
+    const int c = cta + G * j, u = c / cpe, j0 = (c % cpe) * kChunkF;
+    if (!(dist.mask[u] >> tt & 1)) continue;
+    const double* red = s_red + static_cast<size_t>(j) * 16 * T;
+    const double gv = static_cast<double>(xs[tt]) * red[f * T + tt];
+    const double uv = static_cast<double>(xs[tt]) * red[(f + 8) * T + tt];
+    const float hv = static_cast<float>(gv / (1.0 + exp(-gv)) * uv);
+    a.h[(static_cast<size_t>(u) * kMaxTokGemv + tt) * I + j0 + f] = hv;
+    atomicMax(&amax_l[u][tt], __float_as_uint(fabsf(hv)));
+  }
+  __syncthreads();
+  for (int i = tid; i < dist.n * kMaxTokGemv; i += kGUThreads) {
+    const unsigned v = (&amax_l[0][0])[i];
+    if (v) atomicMax(a.amax + i, v);
+  }
 }
 
 // ---------------------------------------------------------- down/combine --
-struct DNSmem {
-  __host__ __device__ static size_t codes(int I) { return align_up(static_cast<size_t>(kNT) * I / 2, 128); }
-  __host__ __device__ static size_t scales(int I) { return align_up(static_cast<size_t>(kNT) * I / 32, 128); }
-  __host__ __device__ static size_t stage(int I) { return codes(I) + scales(I); }
-  __host__ __device__ static size_t act(int I, int T) {
-    return align_up(static_cast<size_t>(T) * (MOE_MAX_TOPK + MOE_MAX_SHARED) * I * 2, 128);
-  }
-  __host__ __device__ static size_t red(int I, int T) { return align_up(static_cast<size_t>(kNT) * (I / 32) * T * 8, 128); }
-  __host__ __device__ static size_t total(int I, int T) { return kStages * stage(I) + act(I, T) + red(I, T); }
+struct DN {
+  // FP8 h of every (expert, token) pair: at most T * (top_k + n_shared) slots
+  __host__ __device__ static size_t act(int I, int slots) { return align_up(static_cast<size_t>(slots) * I, 128); }
+  __host__ __device__ static size_t red(int T) { return kDNWarps * 16 * T * sizeof(double); }
+  __host__ __device__ static size_t total(int I, int T, int slots) { return act(I, slots) + red(T); }
 };
 
-__global__ void down_combine_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kDNThreads)
+down_combine_kernel(GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Distinct dist;
   __shared__ double wsum[kMaxDistinct][kMaxTokGemv];
   __shared__ double coef[kMaxDistinct][kMaxTokGemv];
+  __shared__ float shs[kMaxDistinct][kMaxTokGemv];
   __shared__ int slot_of[kMaxDistinct][kMaxTokGemv];
-  __shared__ __align__(8) uint64_t bars[kStages];
-  __shared__ int s_abort;
+  __shared__ int slot_u[kMaxTokGemv * (MOE_MAX_TOPK + MOE_MAX_SHARED)];
+  __shared__ int slot_t[kMaxTokGemv * (MOE_MAX_TOPK + MOE_MAX_SHARED)];
+  __shared__ int s_nslot;
+  __shared__ int s_ids[kMaxTokGemv * MOE_MAX_TOPK];
+  __shared__ float s_w[kMaxTokGemv * MOE_MAX_TOPK];
+  __shared__ int s_flag;
 
   const int H = a.H, I = a.I, T = a.T;
-  const int tid = threadIdx.x;
-  const int n0 = blockIdx.x * kNT;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int p = blockIdx.x;  // 16-row tile
+  const int n0 = 16 * p;
   const int nb = I / 32;
-  const size_t rowb = I / 2;
+  const size_t tb = tile_bytes(I);
+  const int tiles = H / 16;
+  uint8_t* s_qh = smem;
+  double* s_red = reinterpret_cast<double*>(smem + DN::act(I, T * (a.k + a.n_shared)));
 
-  uint8_t* s_stage = smem;
-  __half* s_act = reinterpret_cast<__half*>(smem + kStages * DNSmem::stage(I));
-  double* s_red = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(s_act) + DNSmem::act(I, T));
-
-  if (tid == 0) {
-    build_distinct(a.ids, a.w, T, a.k, a.E, a.n_shared, dist, wsum, a.err, false);
-    int nslot = 0;
-    for (int u = 0; u < dist.n; ++u)
-      for (int t = 0; t < kMaxTokGemv; ++t) slot_of[u][t] = (t < T && (dist.mask[u] >> t & 1)) ? nslot++ : -1;
-    s_abort = 0;
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-    fence_mbar_init();
-    const uint32_t cb = kNT * rowb, sb = kNT * (I / 32);
-    for (int s = 0; s < kStages && s < dist.n; ++s) {
-      const int e = dist.expert[s];
-      uint8_t* dst = s_stage + s * DNSmem::stage(I);
-      mbar_expect_tx(&bars[s], cb + sb);
-      bulk_g2s(dst, a.w2_codes + (static_cast<size_t>(e) * H + n0) * rowb, cb, &bars[s]);
-      bulk_g2s(dst + DNSmem::codes(I), a.w2_scales + (static_cast<size_t>(e) * H + n0) * (I / 32), sb,
-               &bars[s]);
+  // ---- before the wait: the routing is final (the router grid finished
+  // before the gate/up kernel let this one launch)
+  if (warp == 0) {
+    if (lane < T * a.k) {
+      s_ids[lane] = __ldcg(a.ids + lane);
+      s_w[lane] = __ldcg(a.w + lane);
+    }
+    __syncwarp();
+    build_distinct_warp(s_ids, s_w, T, a.k, a.E, a.n_shared, dist, wsum, a.err, false);
+    if (lane == 0) {
+      int nslot = 0;
+      for (int u = 0; u < dist.n; ++u)
+        for (int t = 0; t < kMaxTokGemv; ++t) {
+          const bool use = t < T && (dist.mask[u] >> t & 1);
+          slot_of[u][t] = use ? nslot : -1;
+          if (use) {
+            slot_u[nslot] = u;
+            slot_t[nslot] = t;
+            ++nslot;
+          }
+        }
+      s_nslot = nslot;
     }
   }
   __syncthreads();
   const int U = dist.n;
+  const int npairs = U * nb;  // (expert, block) pairs, pair q = u * nb + b
+  const int g = lane >> 2, t = lane & 3;
+  // this warp's pairs: warp, warp + 8, ...; the first batch loads now
+  uint2 cw[kDNBatch];
+  uint32_t sc[kDNBatch];
+  auto load = [&](int q0) {
+#pragma unroll
+    for (int i = 0; i < kDNBatch; ++i) {
+      const int q = q0 + i * kDNWarps;
+      if (q < npairs) {
+        const int u = q / nb, b = q % nb;
+        const uint8_t* base = a.w2 + (static_cast<size_t>(dist.expert[u]) * tiles + p) * tb;
+        cw[i] = __ldcs(reinterpret_cast<const uint2*>(base + 256 * b) + lane);
+        sc[i] = __ldcs(reinterpret_cast<const uint16_t*>(base + 256 * nb + 16 * b) + g);
+      }
+    }
+  };
+  load(warp);
 
-  // FP8 activations of every (expert, token) pair -> half, and coefficients
-  for (int u = 0; u < U; ++u) {
-    for (int t = 0; t < T; ++t) {
-      const int sl = slot_of[u][t];
-      if (sl < 0) continue;
-      const uint8_t* q = a.qh + (static_cast<size_t>(u) * kMaxTokGemv + t) * I;
-      for (int j = tid; j < I; j += blockDim.x) s_act[static_cast<size_t>(sl) * I + j] = e4m3_to_half(q[j]);
-      if (tid == 0)
-        coef[u][t] = wsum[u][t] * static_cast<double>(a.sh[static_cast<size_t>(u) * kMaxTokGemv + t]);
+  // ---- after the wait: FP8 re-quantisation of h
+  pdl_wait();
+  const int nslot = s_nslot;
+  if (tid < nslot) {
+    const int u = slot_u[tid], tt = slot_t[tid];
+    const float amax = __uint_as_float(__ldcg(a.amax + u * kMaxTokGemv + tt));
+    const float shv = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+    shs[u][tt] = shv;
+    coef[u][tt] = wsum[u][tt] * static_cast<double>(shv);
+  }
+  // h of every slot, 4 floats per load, 8 loads in flight per thread
+  const int per_slot = I / 4;
+  const int total4 = nslot * per_slot;
+  for (int base = 0; base < total4; base += 8 * kDNThreads) {
+    float4 v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int idx = base + tid + r * kDNThreads;
+      if (idx < total4) {
+        const int sl = idx / per_slot, j4 = idx % per_slot;
+        v[r] = __ldcg(reinterpret_cast<const float4*>(
+                          a.h + (static_cast<size_t>(slot_u[sl]) * kMaxTokGemv + slot_t[sl]) * I) + j4);
+      }
+    }
+    __syncthreads();  // the scales above are visible
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int idx = base + tid + r * kDNThreads;
+      if (idx < total4) {
+        const int sl = idx / per_slot, j = 4 * (idx % per_slot);
+        const float shv = shs[slot_u[sl]][slot_t[sl]];
+        const float hv[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+        uint8_t* row = s_qh + static_cast<size_t>(sl) * I + (j & ~31);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) row[perm_pos((j & 31) + e)] = f32_to_e4m3(__fdiv_rn(hv[e], shv));
+      }
     }
   }
   __syncthreads();
+  // debug copies (one CTA): h, qh, sh per (token, slot)
+  if (blockIdx.x == 0 && (a.dbg.qh || a.dbg.h || a.dbg.sh)) {
+    const int S = a.k + a.n_shared;
+    for (int pp = warp; pp < T * S; pp += kDNWarps) {
+      const int tt = pp / S, si = pp % S;
+      const int e = si < a.k ? s_ids[tt * a.k + si] : a.E + (si - a.k);
+      int u = -1;
+      for (int uu = 0; uu < U; ++uu)
+        if (dist.expert[uu] == e) u = uu;
+      if (u < 0 || slot_of[u][tt] < 0) continue;
+      const int sl = slot_of[u][tt];
+      if (a.dbg.sh && lane == 0) a.dbg.sh[pp] = shs[u][tt];
+      for (int j = lane; j < I; j += 32) {
+        if (a.dbg.qh)
+          a.dbg.qh[static_cast<size_t>(pp) * I + j] = s_qh[static_cast<size_t>(sl) * I + (j & ~31) + perm_pos(j & 31)];
+        if (a.dbg.h) a.dbg.h[static_cast<size_t>(pp) * I + j] =
+            __ldcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + j);
+      }
+    }
+  }
+  // every CTA has read amax: the last one clears it for the next call
+  if (tid == 0) {
+    __threadfence();
+    const int old = atomicAdd(a.down_counter, 1);
+    s_flag = (old == static_cast<int>(gridDim.x) - 1);
+  }
+  __syncthreads();
+  if (s_flag) {
+    for (int i = tid; i < kMaxDistinct * kMaxTokGemv; i += kDNThreads) a.amax[i] = 0u;
+    if (tid == 0) *a.down_counter = 0;
+  }
 
-  const int r = tid / nb, b = tid % nb;
-  const bool active = tid < kNT * nb;
-  double acc[kMaxTokGemv];
+  // ---- tensor-core GEMV over this warp's (expert, block) pairs
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int q0 = warp; q0 < npairs; q0 += kDNBatch * kDNWarps) {
+    if (q0 != warp) load(q0);
 #pragma unroll
-  for (int t = 0; t < kMaxTokGemv; ++t) acc[t] = 0.0;
-
-  for (int u = 0; u < U; ++u) {
-    const int s = u % kStages;
-    if (!mbar_wait_bounded(&bars[s], (u / kStages) & 1, a.err)) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    const uint8_t* st = s_stage + s * DNSmem::stage(I);
-    if (active) {
-      const uint4 c = *reinterpret_cast<const uint4*>(st + static_cast<size_t>(r) * rowb + b * 16);
-      const double f = e8m0_to_f64(st[DNSmem::codes(I) + r * nb + b]);
-#pragma unroll
-      for (int t = 0; t < kMaxTokGemv; ++t) {
-        const int sl = t < T ? slot_of[u][t] : -1;
-        if (sl >= 0) {
-          const uint4* act = reinterpret_cast<const uint4*>(s_act + static_cast<size_t>(sl) * I + b * 32);
-          acc[t] = fma(static_cast<double>(block_dot(c, act)), coef[u][t] * f, acc[t]);
+    for (int i = 0; i < kDNBatch; ++i) {
+      const int q = q0 + i * kDNWarps;
+      if (q < npairs) {
+        const int u = q / nb, b = q % nb;
+        const int slg = g < T ? slot_of[u][g] : -1;
+        uint2 qv = make_uint2(0u, 0u);
+        if (slg >= 0) qv = *reinterpret_cast<const uint2*>(s_qh + static_cast<size_t>(slg) * I + 32 * b + 8 * t);
+        const uint32_t af[4] = {e4m3_lo(cw[i].x), e4m3_lo(cw[i].y), e4m3_hi(cw[i].x), e4m3_hi(cw[i].y)};
+        float d[4];
+        mma_fp8(d, af, qv.x, qv.y);
+        if (2 * t < T) {
+          const double fa = e8m0_to_f64((sc[i] & 0xFFu) + 6), fb = e8m0_to_f64((sc[i] >> 8) + 6);
+          const double c0 = slot_of[u][2 * t] >= 0 ? coef[u][2 * t] : 0.0;
+          acc[0] = fma(static_cast<double>(d[0]), c0 * fa, acc[0]);
+          acc[2] = fma(static_cast<double>(d[2]), c0 * fb, acc[2]);
+          if (2 * t + 1 < T) {
+            const double c1 = slot_of[u][2 * t + 1] >= 0 ? coef[u][2 * t + 1] : 0.0;
+            acc[1] = fma(static_cast<double>(d[1]), c1 * fa, acc[1]);
+            acc[3] = fma(static_cast<double>(d[3]), c1 * fb, acc[3]);
+          }
         }
       }
     }
-    __syncthreads();  // stage s is free again
-    if (tid == 0 && u + kStages < U) {
-      const int e = dist.expert[u + kStages];
-      uint8_t* dst = s_stage + s * DNSmem::stage(I);
-      const uint32_t cb = kNT * rowb, sb = kNT * (I / 32);
-      mbar_expect_tx(&bars[s], cb + sb);
-      bulk_g2s(dst, a.w2_codes + (static_cast<size_t>(e) * H + n0) * rowb, cb, &bars[s]);
-      bulk_g2s(dst + DNSmem::codes(I), a.w2_scales + (static_cast<size_t>(e) * H + n0) * (I / 32), sb,
-               &bars[s]);
+  }
+  if (2 * t < T) {
+    s_red[(warp * 16 + g) * T + 2 * t] = acc[0];
+    s_red[(warp * 16 + g + 8) * T + 2 * t] = acc[2];
+    if (2 * t + 1 < T) {
+      s_red[(warp * 16 + g) * T + 2 * t + 1] = acc[1];
+      s_red[(warp * 16 + g + 8) * T + 2 * t + 1] = acc[3];
     }
   }
-  if (s_abort) {
-    // let copies still in flight land before the CTA's shared memory is released
-    if (tid == 0)
-      for (int u = 0; u < U && u < kStages; ++u) {
-        const int last = u + ((U - 1 - u) / kStages) * kStages;
-        mbar_wait_bounded(&bars[u % kStages], (last / kStages) & 1, nullptr);
-      }
-    return;
-  }
-  if (active)
-    for (int t = 0; t < T; ++t) s_red[(static_cast<size_t>(r) * nb + b) * T + t] = acc[t];
   __syncthreads();
-  if (tid < kNT * T) {
-    const int rr = tid / T, t = tid % T;
-    double s = 0.0;
-    for (int bb = 0; bb < nb; ++bb) s += s_red[(static_cast<size_t>(rr) * nb + bb) * T + t];
-    a.y[static_cast<size_t>(t) * H + n0 + rr] = f64_to_bf16_rne(s);
+  pdl_trigger();
+  if (tid < 16 * T) {
+    const int r = tid / T, tt = tid % T;
+    double sum = 0.0;
+    for (int w = 0; w < kDNWarps; ++w) sum += s_red[(w * 16 + r) * T + tt];
+    a.y[static_cast<size_t>(tt) * H + n0 + r] = f64_to_bf16_rne(sum);
   }
 }
 
 }  // namespace
 
-size_t gemv_workspace_bytes(int I) {
-  const size_t n = static_cast<size_t>(kMaxDistinct) * kMaxTokGemv;
-  return align_up(n * I * 4, 256) + align_up(n * I, 256) + align_up(n * 4, 256) +
-         align_up(kMaxDistinct * 4, 256);
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, Profiler* prof) {
-  const int U_max = a.T * a.k + a.n_shared;
-  const size_t gu_smem = GUSmem::total(a.H, a.T);
-  const size_t dn_smem = DNSmem::total(a.I, a.T);
-  cudaError_t err = cudaFuncSetAttribute(gateup_swiglu_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+int gemv_chunks_per_cta(int I, int T, int k, int n_shared, int n_ctas) {
+  const int chunks = (T * k + n_shared) * (I / kChunkF);
+  return (chunks + n_ctas - 1) / n_ctas;
+}
+
+size_t gemv_smem_bytes(int H, int I, int T, int k, int n_shared, int n_ctas, int which) {
+  return which == 0 ? GU::total(H, T, gemv_chunks_per_cta(I, T, k, n_shared, n_ctas))
+                    : DN::total(I, T, T * (k + n_shared));
+}
+
+cudaError_t launch_gemv(const GemvArgs& a_in, int n_ctas, cudaStream_t stream, Profiler* prof) {
+  GemvArgs a = a_in;
+  a.gu_nmax = gemv_chunks_per_cta(a.I, a.T, a.k, a.n_shared, n_ctas);
+  const size_t gu_smem = GU::total(a.H, a.T, a.gu_nmax);
+  const size_t dn_smem = DN::total(a.I, a.T, a.T * (a.k + a.n_shared));
+  const int nbw = (a.H / 32 + kGUWarps - 1) / kGUWarps;
+  const void* gu = nbw <= 1 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<1>)
+                   : nbw <= 2 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<2>)
+                   : nbw <= 5 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<5>)
+                   : nbw <= 8 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<8>)
+                              : reinterpret_cast<const void*>(gateup_swiglu_kernel<32>);
+  cudaError_t err = cudaFuncSetAttribute(gu, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(gu_smem));
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(dn_smem));
   if (err != cudaSuccess) return err;
+  void* kargs[] = {&a};
   if (prof) prof->before(1, stream);
-  gateup_swiglu_kernel<<<dim3(a.I / kJT, U_max), kGUThreads, gu_smem, stream>>>(a);
-  err = cudaGetLastError();
+  err = launch_pdl(gu, dim3(n_ctas), dim3(kGUThreads), gu_smem, stream, kargs);
   if (prof) prof->after(stream);
   if (err != cudaSuccess) return err;
-  const int threads = (kNT * (a.I / 32) + 31) / 32 * 32;
   if (prof) prof->before(2, stream);
-  down_combine_kernel<<<a.H / kNT, threads, dn_smem, stream>>>(a);
-  err = cudaGetLastError();
+  err = launch_pdl(reinterpret_cast<const void*>(down_combine_kernel), dim3(a.H / 16),
+                   dim3(kDNThreads), dn_smem, stream, kargs);
   if (prof) prof->after(stream);
   return err;
 }

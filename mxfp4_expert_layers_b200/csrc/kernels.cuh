@@ -8,10 +8,29 @@
 
 namespace moe {
 
+// Launch with programmatic stream serialisation (PDL); the kernel's
+// griddepcontrol.wait orders it after the previous kernel of the stream.
+cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       void** args);
+
 // Router (route.cu)
-cudaError_t launch_route(const uint16_t* x, int T, const uint16_t* Wr, const float* bias, int E,
-                         int H, int k, float* logits, int* tile_counter, int* done_counter,
-                         int32_t* ids, float* w, int32_t* counts, cudaStream_t stream);
+struct RouteArgs {
+  int E, H, I, k, n_shared, T;
+  const uint16_t* x;
+  const uint16_t* Wr;
+  const float* bias;
+  float* logits;        // workspace [T][E]
+  int* tile_counter;    // workspace, zero between calls
+  int* done_counter;    // workspace, zero between calls
+  int32_t* ids;
+  float* w;
+  int32_t* counts;
+  // L2 prefetch of the shared experts for the expert kernels that follow
+  int prefetch_shared;
+  const uint8_t* w13;   // packed
+  const uint8_t* w2;    // packed
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 int route_tiles(int T);
 
 // GEMV path, T <= MOE_GEMV_MAX_TOKENS (gemv.cu)
@@ -20,16 +39,15 @@ struct GemvArgs {
   const uint16_t* x;
   const int32_t* ids;
   const float* w;
-  const uint8_t* w13_codes;
-  const uint8_t* w13_scales;
-  const uint8_t* w2_codes;
-  const uint8_t* w2_scales;
+  const uint8_t* w13;   // packed gate/up tiles [E+S][I/8][272 H/32]
+  const uint8_t* w2;    // packed down tiles [E+S][H/16][272 I/32]
   // workspace
-  float* h;             // [kMaxDistinct][kMaxTokGemv][I]
-  uint8_t* qh;          // [kMaxDistinct][kMaxTokGemv][I]
-  float* sh;            // [kMaxDistinct][kMaxTokGemv]
-  int* expert_counter;  // [kMaxDistinct], zero between calls
+  float* h;             // [kMaxDistinct][kMaxTokGemv][I] SwiGLU output
+  unsigned* amax;       // [kMaxDistinct][kMaxTokGemv] float bits of max|h|, zero between calls
+  int* down_counter;    // zero between calls
   int* err;             // device error bits
+  int prefetch_down;    // gate/up CTAs prefetch the down weights into L2
+  int gu_nmax;          // set by launch_gemv: chunks per gate/up CTA at most
   // outputs
   uint16_t* y;          // [T][H]
   moe_debug dbg;
@@ -48,8 +66,22 @@ struct Profiler {
   }
 };
 
-size_t gemv_workspace_bytes(int I);
-cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream, Profiler* prof);
+size_t gemv_smem_bytes(int H, int I, int T, int k, int n_shared, int n_ctas, int which);
+int gemv_chunks_per_cta(int I, int T, int k, int n_shared, int n_ctas);
+
+// Weight packing (pack.cu)
+struct PackArgs {
+  int H, I;
+  int64_t expert0, n_experts;
+  const uint8_t* w13_codes;
+  const uint8_t* w13_scales;
+  const uint8_t* w2_codes;
+  const uint8_t* w2_scales;
+  uint8_t* w13_out;
+  uint8_t* w2_out;
+};
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t stream);
+cudaError_t launch_gemv(const GemvArgs& a, int n_ctas, cudaStream_t stream, Profiler* prof);
 
 // Per-row FP8 quantisation (quant.cu)
 cudaError_t launch_quantize_rows(const float* v, int rows, int cols, uint8_t* q, float* s,

@@ -19,10 +19,10 @@ struct moe_handle_s {
   int* tile_counter;   // [route tiles]
   int* done_counter;   // [1]
   int* err;            // [1]
-  int* expert_counter; // [kMaxDistinct]
+  unsigned* amax;      // [kMaxDistinct][kMaxTokGemv]
+  int* down_counter;   // [1]
   float* h;            // [kMaxDistinct][kMaxTokGemv][I]
-  uint8_t* qh;         // [kMaxDistinct][kMaxTokGemv][I]
-  float* sh;           // [kMaxDistinct][kMaxTokGemv]
+  int n_sms;
   moe::Profiler prof;
   bool profiling;
 };
@@ -69,9 +69,9 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   if (rc) return rc;
   if (max_tokens < 1 || max_tokens > 65536) return MOE_ERR_ARG;
   const moe_weights& w = *weights;
-  if (!w.router_w || !w.w13_codes || !w.w13_scales || !w.w2_codes || !w.w2_scales) return MOE_ERR_ARG;
-  if (!aligned16(w.router_w) || !aligned16(w.w13_codes) || !aligned16(w.w13_scales) ||
-      !aligned16(w.w2_codes) || !aligned16(w.w2_scales) || (w.router_bias && !aligned16(w.router_bias)))
+  if (!w.router_w || !w.w13 || !w.w2) return MOE_ERR_ARG;
+  if (!aligned16(w.router_w) || !aligned16(w.w13) || !aligned16(w.w2) ||
+      (w.router_bias && !aligned16(w.router_bias)))
     return MOE_ERR_ALIGN;
 
   moe_handle h = new (std::nothrow) moe_handle_s();
@@ -83,12 +83,16 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const int E = cfg->n_experts, I = cfg->inter;
   const size_t n_logits = up256(static_cast<size_t>(max_tokens) * E * 4);
   const size_t n_tiles = up256(static_cast<size_t>(moe::route_tiles(max_tokens)) * 4);
-  const size_t n_small = 256;  // done_counter, err
-  const size_t n_ectr = up256(moe::kMaxDistinct * 4);
+  const size_t n_small = 256;  // done_counter, err, down_counter
+  const size_t n_amax = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * I * 4);
-  const size_t n_qh = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * I);
-  const size_t n_sh = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4);
-  h->ws_bytes = n_logits + n_tiles + n_small + n_ectr + n_h + n_qh + n_sh;
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
   if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
     delete h;
     return MOE_ERR_CUDA;
@@ -102,11 +106,10 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->logits = reinterpret_cast<float*>(p); p += n_logits;
   h->tile_counter = reinterpret_cast<int*>(p); p += n_tiles;
   h->done_counter = reinterpret_cast<int*>(p);
-  h->err = reinterpret_cast<int*>(p + 64); p += n_small;
-  h->expert_counter = reinterpret_cast<int*>(p); p += n_ectr;
-  h->h = reinterpret_cast<float*>(p); p += n_h;
-  h->qh = p; p += n_qh;
-  h->sh = reinterpret_cast<float*>(p);
+  h->err = reinterpret_cast<int*>(p + 64);
+  h->down_counter = reinterpret_cast<int*>(p + 128); p += n_small;
+  h->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
+  h->h = reinterpret_cast<float*>(p);
   *out = h;
   return MOE_OK;
 }
@@ -119,10 +122,15 @@ int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* 
       (expert_counts && !aligned4(expert_counts)))
     return MOE_ERR_ALIGN;
   const moe_config& c = h->cfg;
+  moe::RouteArgs a{};
+  a.E = c.n_experts; a.H = c.hidden; a.I = c.inter; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
+  a.x = x; a.Wr = h->w.router_w; a.bias = h->w.router_bias;
+  a.logits = h->logits; a.tile_counter = h->tile_counter; a.done_counter = h->done_counter;
+  a.ids = topk_ids; a.w = topk_w; a.counts = expert_counts;
+  a.prefetch_shared = T <= MOE_GEMV_MAX_TOKENS;
+  a.w13 = h->w.w13; a.w2 = h->w.w2;
   if (h->profiling) h->prof.before(0, stream);
-  const cudaError_t e = moe::launch_route(x, T, h->w.router_w, h->w.router_bias, c.n_experts,
-                                          c.hidden, c.top_k, h->logits, h->tile_counter,
-                                          h->done_counter, topk_ids, topk_w, expert_counts, stream);
+  const cudaError_t e = moe::launch_route(a, stream);
   if (h->profiling) h->prof.after(stream);
   return cuda_err(e);
 }
@@ -137,13 +145,13 @@ int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
   moe::GemvArgs a{};
   a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
   a.x = x; a.ids = topk_ids; a.w = topk_w;
-  a.w13_codes = h->w.w13_codes; a.w13_scales = h->w.w13_scales;
-  a.w2_codes = h->w.w2_codes; a.w2_scales = h->w.w2_scales;
-  a.h = h->h; a.qh = h->qh; a.sh = h->sh; a.expert_counter = h->expert_counter; a.err = h->err;
+  a.w13 = h->w.w13; a.w2 = h->w.w2;
+  a.h = h->h; a.amax = h->amax; a.down_counter = h->down_counter; a.err = h->err;
+  a.prefetch_down = 1;
   a.y = y;
   if (dbg) a.dbg = *dbg;
   h->last_path = 1;
-  return cuda_err(moe::launch_gemv(a, stream, h->profiling ? &h->prof : nullptr));
+  return cuda_err(moe::launch_gemv(a, h->n_sms, stream, h->profiling ? &h->prof : nullptr));
 }
 
 int moe_device_error(moe_handle h, cudaStream_t stream) {
@@ -213,6 +221,23 @@ int moe_destroy(moe_handle h) {
   if (h->ws && cudaFree(h->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
   delete h;
   return rc;
+}
+
+int moe_pack_weights(const moe_config* cfg, const moe_mxfp4_weights* src, int expert0,
+                     int n_experts, uint8_t* w13_packed, uint8_t* w2_packed, cudaStream_t stream) {
+  int rc = validate_config(cfg);
+  if (rc) return rc;
+  if (!src || !w13_packed || !w2_packed || !src->w13_codes || !src->w13_scales || !src->w2_codes ||
+      !src->w2_scales)
+    return MOE_ERR_ARG;
+  if (expert0 < 0 || n_experts < 1 || expert0 + n_experts > cfg->n_experts + cfg->n_shared)
+    return MOE_ERR_ARG;
+  moe::PackArgs a{};
+  a.H = cfg->hidden; a.I = cfg->inter; a.expert0 = expert0; a.n_experts = n_experts;
+  a.w13_codes = src->w13_codes; a.w13_scales = src->w13_scales;
+  a.w2_codes = src->w2_codes; a.w2_scales = src->w2_scales;
+  a.w13_out = w13_packed; a.w2_out = w2_packed;
+  return cuda_err(moe::launch_pack(a, stream));
 }
 
 int moe_quantize_fp8(const float* v, int rows, int cols, uint8_t* q, float* s,

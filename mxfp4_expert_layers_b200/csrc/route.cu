@@ -5,11 +5,14 @@
 // MoE layer).  Scoring (softmax over float32 logits, top-k, renormalised)
 // and the float64 accumulation of the logits are this library's reading.
 //
-// One launch.  Grid (ceil(E / 4), ceil(T / kTokTile)); each warp computes
-// the logits of one expert for the CTA's tokens and stores them in the
-// workspace.  The last CTA of a token tile to finish (atomic counter, no
-// waiting) selects the top-k of those tokens; the last token tile to finish
-// builds the per-expert counts.  Counters reset themselves for the next call.
+// One launch.  Grid (ceil(E / 4), ceil(T / kTokTile)); each warp owns one
+// expert row.  Before its dependency wait (programmatic dependent launch) a
+// warp loads its router row into registers and the first CTAs prefetch the
+// shared experts' weights into L2; after the wait it reads x (the previous
+// kernel's output) and accumulates the logits: bf16 x bf16 products are exact
+// in float32 and are summed in float64.  The last CTA of a token tile to
+// finish (atomic counter, no waiting) selects the top-k of those tokens; the
+// last token tile builds the per-expert counts.  Counters reset themselves.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -24,7 +27,8 @@ __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
   return a > b || (a == b && ia < ib);
 }
 
-// Top-k of one token's logits by one warp; lane 0 writes ids and weights.
+// Top-k of one token's logits by one warp.  Lane r keeps the r-th selection;
+// the softmax over the selected logits runs on lanes 0..k-1 in float64.
 __device__ void warp_topk(const float* logits, int E, int k, int32_t* ids_out,
                           float* w_out) {
   const int lane = threadIdx.x & 31;
@@ -36,8 +40,8 @@ __device__ void warp_topk(const float* logits, int E, int k, int32_t* ids_out,
     const int e = lane + 32 * i;
     v[i] = e < E ? __ldcg(logits + e) : 0.f;
   }
-  float sel[MOE_MAX_TOPK];
-  int sid[MOE_MAX_TOPK];
+  float my_sel = 0.f;
+  int my_id = -1;
   for (int r = 0; r < k; ++r) {
     float bv = 0.f;
     int bi = -1;
@@ -58,64 +62,102 @@ __device__ void warp_topk(const float* logits, int E, int k, int32_t* ids_out,
       }
     }
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    sel[r] = bv;
-    sid[r] = bi;
+    if (lane == r) {
+      my_sel = bv;
+      my_id = bi;
+    }
   }
-  if (lane == 0) {
-    // softmax over the selected logits in float64; sel[0] is the largest
-    double z[MOE_MAX_TOPK];
-    double sum = 0.0;
-    for (int r = 0; r < k; ++r) {
-      z[r] = exp(static_cast<double>(sel[r]) - static_cast<double>(sel[0]));
-      sum += z[r];
-    }
-    for (int r = 0; r < k; ++r) {
-      ids_out[r] = sid[r];
-      w_out[r] = static_cast<float>(z[r] / sum);
-    }
+  // softmax over the selected logits; the first selection is the largest
+  const double top = static_cast<double>(__shfl_sync(0xffffffffu, my_sel, 0));
+  const double z = lane < k ? exp(static_cast<double>(my_sel) - top) : 0.0;
+  const double sum = warp_sum_f64(z);
+  if (lane < k) {
+    ids_out[lane] = my_id;
+    w_out[lane] = static_cast<float>(z / sum);
   }
 }
 
+__device__ __forceinline__ void bf16x2_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+// acc += sum of the 8 exact float32 products of two 16-byte chunks
+__device__ __forceinline__ double dot8(const uint4 wv, const uint4 xv, double acc) {
+  const uint32_t wp[4] = {wv.x, wv.y, wv.z, wv.w};
+  const uint32_t xp[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float w0, w1, x0, x1;
+    bf16x2_f32(wp[j], w0, w1);
+    bf16x2_f32(xp[j], x0, x1);
+    acc += static_cast<double>(__fmul_rn(w0, x0));
+    acc += static_cast<double>(__fmul_rn(w1, x1));
+  }
+  return acc;
+}
+
+// NCH = 16-byte chunks of a router row per lane kept in registers (0: rows
+// longer than 16 chunks per lane, streamed from global memory instead).
+template <int NCH>
 __global__ void __launch_bounds__(kWarps * 32)
-route_kernel(const uint16_t* __restrict__ x, int T, const uint16_t* __restrict__ Wr,
-             const float* __restrict__ bias, int E, int H, int k, float* __restrict__ logits,
-             int* __restrict__ tile_counter, int* __restrict__ done_counter,
-             int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ counts) {
+route_kernel(RouteArgs a) {
+  constexpr int kRegChunks = NCH;
   __shared__ int s_last;
   __shared__ int s_hist[MOE_MAX_EXPERTS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E, H = a.H, T = a.T;
   const int e = blockIdx.x * kWarps + warp;
   const int t0 = blockIdx.y * kTokTile;
   const int nt = min(kTokTile, T - t0);
+  const int nchunk = H / 8;  // 8 bf16 per 16 bytes
+
+  // ---- before the wait: router row into registers; shared experts into L2
+  uint4 wreg[kRegChunks > 0 ? kRegChunks : 1];
+  const uint4* wrow = reinterpret_cast<const uint4*>(a.Wr + static_cast<size_t>(e < E ? e : 0) * H);
+#pragma unroll
+  for (int i = 0; i < kRegChunks; ++i) {
+    const int c = lane + 32 * i;
+    wreg[i] = (e < E && c < nchunk) ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (a.prefetch_shared && blockIdx.y == 0 && threadIdx.x == 0) {
+    // shared experts' packed gate/up and down weights (each expert
+    // contiguous), sliced over the CTAs
+    const size_t n13 = static_cast<size_t>(a.I / 8) * 272 * (H / 32);
+    const size_t n2 = static_cast<size_t>(H / 16) * 272 * (a.I / 32);
+    const uint8_t* parts[2] = {a.w13 + static_cast<size_t>(E) * n13, a.w2 + static_cast<size_t>(E) * n2};
+    const size_t sizes[2] = {a.n_shared * n13, a.n_shared * n2};
+    for (int q = 0; q < 2; ++q) {
+      const size_t s0 = (sizes[q] * blockIdx.x / gridDim.x) & ~static_cast<size_t>(15);
+      const size_t s1 = (sizes[q] * (blockIdx.x + 1) / gridDim.x) & ~static_cast<size_t>(15);
+      if (s1 > s0) prefetch_l2(parts[q] + s0, static_cast<uint32_t>(s1 - s0));
+    }
+  }
+
+  pdl_wait();
+  pdl_trigger();
 
   if (e < E) {
     double acc[kTokTile];
 #pragma unroll
     for (int t = 0; t < kTokTile; ++t) acc[t] = 0.0;
-    const uint4* wrow = reinterpret_cast<const uint4*>(Wr + static_cast<size_t>(e) * H);
-    const int nchunk = H / 8;  // 8 bf16 per 16 bytes
-    for (int c = lane; c < nchunk; c += 32) {
-      const uint4 wv = __ldg(wrow + c);
-      const uint32_t wp[4] = {wv.x, wv.y, wv.z, wv.w};
-      double wd[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        wd[2 * j] = bf16_bits_to_f32(static_cast<uint16_t>(wp[j] & 0xFFFF));
-        wd[2 * j + 1] = bf16_bits_to_f32(static_cast<uint16_t>(wp[j] >> 16));
-      }
+    for (int t = 0; t < kTokTile; ++t) {
+      if (t < nt) {
+        const uint4* xrow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + t) * H);
+        if (kRegChunks > 0) {
+          uint4 xr[kRegChunks > 0 ? kRegChunks : 1];
 #pragma unroll
-      for (int t = 0; t < kTokTile; ++t) {
-        if (t < nt) {
-          const uint4 xv =
-              __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + t) * H) + c);
-          const uint32_t xp[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            acc[t] = fma(static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xp[j] & 0xFFFF))),
-                         wd[2 * j], acc[t]);
-            acc[t] = fma(static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xp[j] >> 16))),
-                         wd[2 * j + 1], acc[t]);
+          for (int i = 0; i < kRegChunks; ++i) {  // all loads first, then the arithmetic
+            const int c = lane + 32 * i;
+            xr[i] = c < nchunk ? __ldcg(xrow + c) : make_uint4(0u, 0u, 0u, 0u);
           }
+          double part[4] = {0.0, 0.0, 0.0, 0.0};  // exact partial sums, any order
+#pragma unroll
+          for (int i = 0; i < kRegChunks; ++i) part[i & 3] = dot8(wreg[i], xr[i], part[i & 3]);
+          acc[t] = (part[0] + part[1]) + (part[2] + part[3]);
+        } else {
+          for (int c = lane; c < nchunk; c += 32) acc[t] = dot8(__ldg(wrow + c), __ldcg(xrow + c), acc[t]);
         }
       }
     }
@@ -125,8 +167,8 @@ route_kernel(const uint16_t* __restrict__ x, int T, const uint16_t* __restrict__
         const double s = warp_sum_f64(acc[t]);
         if (lane == 0) {
           float l = static_cast<float>(s);
-          if (bias) l = __fadd_rn(l, bias[e]);
-          logits[static_cast<size_t>(t0 + t) * E + e] = l;
+          if (a.bias) l = __fadd_rn(l, a.bias[e]);
+          a.logits[static_cast<size_t>(t0 + t) * E + e] = l;
         }
       }
     }
@@ -136,20 +178,20 @@ route_kernel(const uint16_t* __restrict__ x, int T, const uint16_t* __restrict__
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int old = atomicAdd(&tile_counter[blockIdx.y], 1);
+    const int old = atomicAdd(&a.tile_counter[blockIdx.y], 1);
     s_last = (old == static_cast<int>(gridDim.x) - 1);
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
   for (int t = warp; t < nt; t += kWarps)
-    warp_topk(logits + static_cast<size_t>(t0 + t) * E, E, k,
-              ids + static_cast<size_t>(t0 + t) * k, w + static_cast<size_t>(t0 + t) * k);
+    warp_topk(a.logits + static_cast<size_t>(t0 + t) * E, E, a.k,
+              a.ids + static_cast<size_t>(t0 + t) * a.k, a.w + static_cast<size_t>(t0 + t) * a.k);
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    tile_counter[blockIdx.y] = 0;
-    const int old = atomicAdd(done_counter, 1);
+    a.tile_counter[blockIdx.y] = 0;
+    const int old = atomicAdd(a.done_counter, 1);
     s_last = (old == static_cast<int>(gridDim.y) - 1);
   }
   __syncthreads();
@@ -158,25 +200,29 @@ route_kernel(const uint16_t* __restrict__ x, int T, const uint16_t* __restrict__
   __threadfence();
   for (int i = threadIdx.x; i < E; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-    const int id = __ldcg(ids + i);
+  for (int i = threadIdx.x; i < T * a.k; i += blockDim.x) {
+    const int id = __ldcg(a.ids + i);
     if (id >= 0 && id < E) atomicAdd(&s_hist[id], 1);
   }
   __syncthreads();
-  if (counts)
-    for (int i = threadIdx.x; i < E; i += blockDim.x) counts[i] = s_hist[i];
-  if (threadIdx.x == 0) *done_counter = 0;
+  if (a.counts)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) a.counts[i] = s_hist[i];
+  if (threadIdx.x == 0) *a.done_counter = 0;
 }
 
 }  // namespace
 
-cudaError_t launch_route(const uint16_t* x, int T, const uint16_t* Wr, const float* bias, int E,
-                         int H, int k, float* logits, int* tile_counter, int* done_counter,
-                         int32_t* ids, float* w, int32_t* counts, cudaStream_t stream) {
-  dim3 grid((E + kWarps - 1) / kWarps, (T + kTokTile - 1) / kTokTile);
-  route_kernel<<<grid, kWarps * 32, 0, stream>>>(x, T, Wr, bias, E, H, k, logits, tile_counter,
-                                                 done_counter, ids, w, counts);
-  return cudaGetLastError();
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
+  dim3 grid((a.E + kWarps - 1) / kWarps, (a.T + kTokTile - 1) / kTokTile);
+  RouteArgs args = a;
+  void* kargs[] = {&args};
+  const int need = (a.H / 8 + 31) / 32;
+  const void* fn = need <= 2    ? reinterpret_cast<const void*>(route_kernel<2>)
+                   : need <= 4  ? reinterpret_cast<const void*>(route_kernel<4>)
+                   : need <= 10 ? reinterpret_cast<const void*>(route_kernel<10>)
+                   : need <= 16 ? reinterpret_cast<const void*>(route_kernel<16>)
+                                : reinterpret_cast<const void*>(route_kernel<0>);
+  return launch_pdl(fn, grid, dim3(kWarps * 32), 0, stream, kargs);
 }
 
 int route_tiles(int T) { return (T + kTokTile - 1) / kTokTile; }

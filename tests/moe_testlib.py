@@ -49,6 +49,7 @@ class GpuLayer:
         self.seed, self.layer, self.E, self.H, self.I, self.k, self.S = seed, layer, E, H, I, k, n_shared
         n = E + n_shared
         dev = "cuda"
+        self.canon = {}
         if weights is None:
             self.t = {
                 "router_w": torch.empty((E, H), dtype=torch.int16, device=dev),
@@ -77,7 +78,14 @@ class GpuLayer:
             b = synth.zipf_router_bias(seed, layer, E) if bias is True else np.asarray(bias, np.float32)
             self.t["router_bias"] = to_dev(b)
             self.host.router_bias = b
+        # packed layout the kernels read
+        self.t["w13"] = torch.empty((n, I // 8, moe.w13_tile_bytes(H)), dtype=torch.uint8, device=dev)
+        self.t["w2"] = torch.empty((n, H // 16, moe.w2_tile_bytes(I)), dtype=torch.uint8, device=dev)
+        moe.moe_pack_weights(H, I, E, k, n_shared, self.t, 0, n, self.t["w13"], self.t["w2"])
         torch.cuda.synchronize()
+        for key in ("w13_codes", "w13_scales", "w2_codes", "w2_scales"):
+            self.canon = getattr(self, "canon", {})
+            self.canon[key] = self.t.pop(key)
         self.handle = moe.moe_create(H, I, E, k, n_shared, self.t, max_tokens)
 
     def close(self):

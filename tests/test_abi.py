@@ -40,8 +40,7 @@ def test_strerror_names_every_code():
 
 
 def _weights(ptr=0x1000):
-    return {"router_w": ptr, "router_bias": None, "w13_codes": ptr, "w13_scales": ptr,
-            "w2_codes": ptr, "w2_scales": ptr}
+    return {"router_w": ptr, "router_bias": None, "w13": ptr, "w2": ptr}
 
 
 @pytest.mark.parametrize("cfg,code", [
@@ -62,7 +61,7 @@ def test_create_validates_shapes(cfg, code):
 
 def test_create_rejects_null_and_bad_token_count():
     w = _weights(0x1000)
-    w["w2_codes"] = None
+    w["w2"] = None
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_create(2560, 768, 512, 8, 1, w, 4)
     assert ei.value.code == moe.MOE_ERR_ARG

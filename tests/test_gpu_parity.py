@@ -46,7 +46,46 @@ def test_gpu_fill_matches_host_generator():
         for e in (0, 7, E):                          # includes the shared expert
             ref = synth.expert_weights(5, 3, e, H, I)
             for key in ref:
-                assert np.array_equal(L.t[key][e].cpu().numpy(), ref[key]), (e, key)
+                assert np.array_equal(L.canon[key][e].cpu().numpy(), ref[key]), (e, key)
+    finally:
+        L.close()
+
+
+def _pack_tiles_numpy(codes, scales, row_a, row_b):
+    """Packed tile bytes written out from the layout's definition: per block
+    b, lane L = 4g+t: bytes 16b+4t.. of rows row_a(g) and row_b(g); then per
+    block the scale pairs (row_a(g), row_b(g))."""
+    nb = scales.shape[1]
+    out = []
+    for b in range(nb):
+        for L in range(32):
+            g, t = L // 4, L % 4
+            out.append(codes[row_a(g), 16 * b + 4 * t:16 * b + 4 * t + 4])
+            out.append(codes[row_b(g), 16 * b + 4 * t:16 * b + 4 * t + 4])
+    for b in range(nb):
+        for g in range(8):
+            out.append(np.array([scales[row_a(g), b], scales[row_b(g), b]], np.uint8))
+    return np.concatenate(out)
+
+
+def test_gpu_pack_layout_matches_definition():
+    E, H, I = 8, 256, 128
+    L = GpuLayer(6, 1, E, H, I, k=2, fill="gpu")
+    try:
+        w13 = L.t["w13"].cpu().numpy()
+        w2 = L.t["w2"].cpu().numpy()
+        for e in (0, 5, E):
+            ex = synth.expert_weights(6, 1, e, H, I)
+            for c in (0, 3, I // 8 - 1):
+                want = _pack_tiles_numpy(ex["w13_codes"], ex["w13_scales"],
+                                         lambda g: 8 * c + g, lambda g: I + 8 * c + g)
+                assert np.array_equal(w13[e, c], want), (e, c)
+            for pt in (0, 7, H // 16 - 1):
+                want = _pack_tiles_numpy(ex["w2_codes"], ex["w2_scales"],
+                                         lambda g: 16 * pt + g, lambda g: 16 * pt + 8 + g)
+                assert np.array_equal(w2[e, pt], want), (e, pt)
+        # a permutation: every byte accounted for
+        assert w13.size == L.canon["w13_codes"].numel() + L.canon["w13_scales"].numel()
     finally:
         L.close()
 
