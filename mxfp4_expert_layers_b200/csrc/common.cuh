@@ -16,6 +16,25 @@
 
 namespace moe {
 
+// Phase timestamps for timeline analysis: compiled in only with -DMOE_TRACE
+// (thread 0 of each CTA writes %globaltimer to a per-file table); nothing
+// otherwise.
+#ifdef MOE_TRACE
+static __device__ unsigned long long g_trace[4][512][64];
+#define MOE_TRACE_POINT(k, slot)                                                    \
+  do {                                                                              \
+    if (threadIdx.x == 0) {                                                         \
+      unsigned long long t_;                                                        \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                        \
+      g_trace[k][blockIdx.x + gridDim.x * blockIdx.y][slot] = t_;                   \
+    }                                                                               \
+  } while (0)
+#else
+#define MOE_TRACE_POINT(k, slot) \
+  do {                           \
+  } while (0)
+#endif
+
 // ----------------------------------------------------------------- limits --
 constexpr int kBlockK = 32;               // MX block along K
 constexpr int kMaxSlots = MOE_MAX_TOPK + MOE_MAX_SHARED;

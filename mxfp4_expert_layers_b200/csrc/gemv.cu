@@ -42,7 +42,8 @@ constexpr int kGUWarps = kGUThreads / 32;
 constexpr int kDNThreads = 256;   // 8 warps
 constexpr int kDNWarps = kDNThreads / 32;
 constexpr int kChunkF = 8;        // features per chunk (16 rows with gate + up)
-constexpr int kDNBatch = 28;      // (expert, block) pairs per warp held in registers
+constexpr int kGUMaxStages = 8;   // chunk stages per gate/up CTA
+constexpr int kDNMaxStages = 12;  // expert slabs per down CTA
 
 __host__ __device__ constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 __host__ __device__ constexpr size_t tile_bytes(int K) { return 272u * static_cast<size_t>(K / 32); }
@@ -88,6 +89,10 @@ __device__ void build_distinct_warp(const int32_t* ids, const float* w, int T, i
   __syncwarp();
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 8 E2M1 codes (one word) -> E4M3 bytes holding value * 2^-6: the codes of
 // the high nibbles (elements 1, 3, 5, 7) and of the low nibbles (0, 2, 4, 6)
 __device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) { return (w & 0x80808080u) | ((w & 0x70707070u) >> 2); }
@@ -118,27 +123,58 @@ struct GU {
   __host__ __device__ static size_t red(int T, int nmax) {
     return align_up(static_cast<size_t>(nmax) * 16 * T * sizeof(double), 128);
   }
-  __host__ __device__ static size_t total(int H, int T, int nmax) { return act(H, T) + red(T, nmax); }
+  __host__ __device__ static size_t stage(int H) { return align_up(tile_bytes(H), 128); }
+  __host__ __device__ static size_t total(int H, int T, int nmax, int ns) {
+    return ns * stage(H) + act(H, T) + red(T, nmax);
+  }
+  // all of a CTA's chunks in flight when they fit, else a ring
+  static int stages(int H, int T, int nmax) {
+    int ns = nmax < kGUMaxStages ? nmax : kGUMaxStages;
+    if (ns < 1) ns = 1;
+    while (ns > 2 && total(H, T, nmax, ns) > 150 * 1024) --ns;
+    return ns;
+  }
 };
 
-template <int NBW>  // blocks per warp per chunk: ceil((H/32) / 16)
+__device__ __forceinline__ void gu_issue(const GemvArgs& a, int e, int cin, uint8_t* st, uint64_t* bar) {
+  const uint32_t tb = static_cast<uint32_t>(tile_bytes(a.H));
+  mbar_expect_tx(bar, tb);
+  bulk_g2s(st, a.w13 + (static_cast<size_t>(e) * (a.I / kChunkF) + cin) * tb, tb, bar);
+}
+
 __global__ void __launch_bounds__(kGUThreads)
 gateup_swiglu_kernel(GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Distinct dist;
   __shared__ double wsum[kMaxDistinct][kMaxTokGemv];
+  __shared__ __align__(8) uint64_t full[kGUMaxStages];
+  __shared__ __align__(8) uint64_t empty[kGUMaxStages];
   __shared__ float red_f[kGUWarps];
   __shared__ float xs[kMaxTokGemv];
   __shared__ int s_ids[kMaxTokGemv * MOE_MAX_TOPK];
   __shared__ unsigned amax_l[kMaxDistinct][kMaxTokGemv];
+  __shared__ int s_abort;
 
-  const int H = a.H, I = a.I, T = a.T;
+  const int H = a.H, I = a.I, T = a.T, NS = a.gu_stages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int cpe = I / kChunkF, nb = H / 32;
-  uint8_t* s_act = smem;                                            // [T][H] permuted E4M3
-  double* s_red = reinterpret_cast<double*>(smem + GU::act(H, T));  // [chunk][16][T]
+  uint8_t* s_stage = smem;
+  uint8_t* s_act = smem + NS * GU::stage(H);                          // [T][H] permuted E4M3
+  double* s_red = reinterpret_cast<double*>(s_act + GU::act(H, T));   // [chunk][16][T]
 
+  MOE_TRACE_POINT(1, 0);
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGUWarps);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+    // the CTA's first chunk belongs to a shared expert when cta < n_shared * I/8:
+    // its copy starts before the routing is known
+    if (cta < a.n_shared * cpe) gu_issue(a, a.E + cta / cpe, cta % cpe, s_stage, &full[0]);
+  }
   for (int i = tid; i < kMaxDistinct * kMaxTokGemv; i += kGUThreads) (&amax_l[0][0])[i] = 0u;
   for (int i = tid; i < a.gu_nmax * 16 * T; i += kGUThreads) s_red[i] = 0.0;
 
@@ -206,8 +242,10 @@ gateup_swiglu_kernel(GemvArgs a) {
     }
   }
 
+  MOE_TRACE_POINT(1, 1);
   // ---- routing of this call (written by the router kernel)
   pdl_wait();
+  MOE_TRACE_POINT(1, 2);
   if (warp == 0) {
     if (lane < T * a.k) s_ids[lane] = __ldcg(a.ids + lane);
     __syncwarp();
@@ -216,8 +254,15 @@ gateup_swiglu_kernel(GemvArgs a) {
   __syncthreads();
   pdl_trigger();
 
+  MOE_TRACE_POINT(1, 3);
   const int nchunks = dist.n * cpe;
   const int nmine = cta < nchunks ? (nchunks - 1 - cta) / G + 1 : 0;
+  if (tid == 0)
+    for (int j = 0; j < NS && j < nmine; ++j) {
+      const int c = cta + G * j;
+      if (c < a.n_shared * cpe && j == 0) continue;  // already in flight
+      gu_issue(a, dist.expert[c / cpe], c % cpe, s_stage + j * GU::stage(H), &full[j]);
+    }
   // L2 prefetch of the down weights this call needs: CTA b takes a slice of
   // every expert's packed down weights
   if (warp == 1 && a.prefetch_down) {
@@ -230,53 +275,39 @@ gateup_swiglu_kernel(GemvArgs a) {
   }
 
   const int g = lane >> 2, t = lane & 3;
-  const int bw0 = warp * NBW;
-  const size_t tb = tile_bytes(H);
-  // fragments of one chunk: word pairs and scale pairs of this lane's blocks
-  uint2 cw[2][NBW];
-  uint32_t sc[2][NBW];
-  auto load = [&](int j, int buf) {
-    const int c = cta + G * j;
-    const uint8_t* base = a.w13 + (static_cast<size_t>(dist.expert[c / cpe]) * cpe + c % cpe) * tb;
-#pragma unroll
-    for (int i = 0; i < NBW; ++i) {
-      const int b = bw0 + i;
-      if (b < nb) {
-        cw[buf][i] = __ldcs(reinterpret_cast<const uint2*>(base + 256 * b) + lane);
-        sc[buf][i] = __ldcs(reinterpret_cast<const uint16_t*>(base + 256 * nb + 16 * b) + g);
-      }
-    }
-  };
-  auto compute = [&](int j, int buf) {
-    const int c = cta + G * j;
+  const int nbw = (nb + kGUWarps - 1) / kGUWarps;
+  const int b0 = warp * nbw, b1 = min(nb, b0 + nbw);
+  for (int j = 0; j < nmine; ++j) {
+    const int c = cta + G * j, s = j % NS;
+    const uint8_t* st = s_stage + s * GU::stage(H);
+    if (!mbar_wait_bounded(&full[s], (j / NS) & 1, a.err)) s_abort = 1;
+    if (*reinterpret_cast<volatile int*>(&s_abort)) break;
+    if (j < 16) MOE_TRACE_POINT(1, 8 + j);
     const int u = c / cpe;
-    const unsigned mask = dist.mask[u];
-    const bool tok = g < T && (mask >> g & 1);
+    const bool tok = g < T && (dist.mask[u] >> g & 1);
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-    for (int i = 0; i < NBW; ++i) {
-      const int b = bw0 + i;
-      if (b < nb) {
-        const uint32_t wa = cw[buf][i].x, wb = cw[buf][i].y;
-        const uint32_t af[4] = {e4m3_lo(wa), e4m3_lo(wb), e4m3_hi(wa), e4m3_hi(wb)};
-        uint2 q = make_uint2(0u, 0u);
-        if (tok) q = *reinterpret_cast<const uint2*>(s_act + static_cast<size_t>(g) * H + 32 * b + 8 * t);
-        float d[4];
-        mma_fp8(d, af, q.x, q.y);
-        if (2 * t < T) {
-          const double fa = e8m0_to_f64((sc[buf][i] & 0xFFu) + 6), fb = e8m0_to_f64((sc[buf][i] >> 8) + 6);
-          acc[0] = fma(static_cast<double>(d[0]), fa, acc[0]);
-          acc[2] = fma(static_cast<double>(d[2]), fb, acc[2]);
-          if (2 * t + 1 < T) {
-            acc[1] = fma(static_cast<double>(d[1]), fa, acc[1]);
-            acc[3] = fma(static_cast<double>(d[3]), fb, acc[3]);
-          }
+#pragma unroll 5
+    for (int b = b0; b < b1; ++b) {
+      const uint2 cw = *reinterpret_cast<const uint2*>(st + 256 * b + 8 * lane);
+      const uint32_t sc = *reinterpret_cast<const uint16_t*>(st + 256 * nb + 16 * b + 2 * g);
+      const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+      uint2 q = make_uint2(0u, 0u);
+      if (tok) q = *reinterpret_cast<const uint2*>(s_act + static_cast<size_t>(g) * H + 32 * b + 8 * t);
+      float d[4];
+      mma_fp8(d, af, q.x, q.y);
+      if (2 * t < T) {
+        const double fa = e8m0_to_f64((sc & 0xFFu) + 6), fb = e8m0_to_f64((sc >> 8) + 6);
+        acc[0] = fma(static_cast<double>(d[0]), fa, acc[0]);
+        acc[2] = fma(static_cast<double>(d[2]), fb, acc[2]);
+        if (2 * t + 1 < T) {
+          acc[1] = fma(static_cast<double>(d[1]), fa, acc[1]);
+          acc[3] = fma(static_cast<double>(d[3]), fb, acc[3]);
         }
       }
     }
     // exact partial sums: order-free float64 atomics
     double* red = s_red + static_cast<size_t>(j) * 16 * T;
-    if (2 * t < T && bw0 < nb) {
+    if (2 * t < T && b0 < nb) {
       atomicAdd(&red[g * T + 2 * t], acc[0]);
       atomicAdd(&red[(g + 8) * T + 2 * t], acc[2]);
       if (2 * t + 1 < T) {
@@ -284,15 +315,30 @@ gateup_swiglu_kernel(GemvArgs a) {
         atomicAdd(&red[(g + 8) * T + 2 * t + 1], acc[3]);
       }
     }
-  };
-  if (nmine > 0) load(0, 0);
-  for (int j = 0; j < nmine; j += 2) {
-    if (j + 1 < nmine) load(j + 1, 1);
-    compute(j, 0);
-    if (j + 2 < nmine) load(j + 2, 0);
-    if (j + 1 < nmine) compute(j + 1, 1);
+    // release the stage; warp 0 refills it with the CTA's chunk j + NS
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (warp == 0 && j + NS < nmine) {
+      if (!mbar_wait_bounded(&empty[s], (j / NS) & 1, a.err)) {
+        s_abort = 1;
+      } else if (lane == 0) {
+        const int cn = cta + G * (j + NS);
+        gu_issue(a, dist.expert[cn / cpe], cn % cpe, s_stage + s * GU::stage(H), &full[s]);
+      }
+      __syncwarp();
+    }
   }
   __syncthreads();
+  if (s_abort) {
+    // let the copies still in flight land before the CTA exits (bounded)
+    if (tid == 0)
+      for (int s = 0; s < NS; ++s) {
+        mbar_wait_bounded(&full[s], 0, nullptr);
+        mbar_wait_bounded(&full[s], 1, nullptr);
+      }
+    return;
+  }
+  MOE_TRACE_POINT(1, 4);
   // SwiGLU of every feature of every chunk of this CTA
   for (int p = tid; p < nmine * kChunkF * T; p += kGUThreads) {
     const int j = p / (kChunkF * T), r = p % (kChunkF * T), f = r / T, tt = r % T;
@@ -310,6 +356,7 @@ gateup_swiglu_kernel(GemvArgs a) {
     const unsigned v = (&amax_l[0][0])[i];
     if (v) atomicMax(a.amax + i, v);
   }
+  MOE_TRACE_POINT(1, 5);
 }
 
 // ---------------------------------------------------------- down/combine --
@@ -317,8 +364,18 @@ struct DN {
   // FP8 h of every (expert, token) pair: at most T * (top_k + n_shared) slots
   __host__ __device__ static size_t act(int I, int slots) { return align_up(static_cast<size_t>(slots) * I, 128); }
   __host__ __device__ static size_t red(int T) { return kDNWarps * 16 * T * sizeof(double); }
-  __host__ __device__ static size_t total(int I, int T, int slots) { return act(I, slots) + red(T); }
+  __host__ __device__ static size_t stage(int I) { return align_up(tile_bytes(I), 128); }
+  __host__ __device__ static int stages(int U) { return U < kDNMaxStages ? U : kDNMaxStages; }
+  __host__ __device__ static size_t total(int I, int T, int U, int slots) {
+    return stages(U) * stage(I) + act(I, slots) + red(T);
+  }
 };
+
+__device__ __forceinline__ void dn_issue(const GemvArgs& a, int e, int p, uint8_t* st, uint64_t* bar) {
+  const uint32_t tb = static_cast<uint32_t>(tile_bytes(a.I));
+  mbar_expect_tx(bar, tb);
+  bulk_g2s(st, a.w2 + (static_cast<size_t>(e) * (a.H / 16) + p) * tb, tb, bar);
+}
 
 __global__ void __launch_bounds__(kDNThreads)
 down_combine_kernel(GemvArgs a) {
@@ -333,20 +390,24 @@ down_combine_kernel(GemvArgs a) {
   __shared__ int s_nslot;
   __shared__ int s_ids[kMaxTokGemv * MOE_MAX_TOPK];
   __shared__ float s_w[kMaxTokGemv * MOE_MAX_TOPK];
+  __shared__ __align__(8) uint64_t bars[kDNMaxStages];
   __shared__ int s_flag;
+  __shared__ int s_abort;
 
   const int H = a.H, I = a.I, T = a.T;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int p = blockIdx.x;  // 16-row tile
-  const int n0 = 16 * p;
-  const int nb = I / 32;
-  const size_t tb = tile_bytes(I);
+  const int G = gridDim.x;
   const int tiles = H / 16;
-  uint8_t* s_qh = smem;
-  double* s_red = reinterpret_cast<double*>(smem + DN::act(I, T * (a.k + a.n_shared)));
+  const int nb = I / 32;
 
   // ---- before the wait: the routing is final (the router grid finished
-  // before the gate/up kernel let this one launch)
+  // before the gate/up kernel let this one launch); start the weight copies
+  MOE_TRACE_POINT(2, 0);
+  if (tid == 0) {
+    for (int s = 0; s < kDNMaxStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
   if (warp == 0) {
     if (lane < T * a.k) {
       s_ids[lane] = __ldcg(a.ids + lane);
@@ -371,27 +432,21 @@ down_combine_kernel(GemvArgs a) {
   }
   __syncthreads();
   const int U = dist.n;
-  const int npairs = U * nb;  // (expert, block) pairs, pair q = u * nb + b
-  const int g = lane >> 2, t = lane & 3;
-  // this warp's pairs: warp, warp + 8, ...; the first batch loads now
-  uint2 cw[kDNBatch];
-  uint32_t sc[kDNBatch];
-  auto load = [&](int q0) {
-#pragma unroll
-    for (int i = 0; i < kDNBatch; ++i) {
-      const int q = q0 + i * kDNWarps;
-      if (q < npairs) {
-        const int u = q / nb, b = q % nb;
-        const uint8_t* base = a.w2 + (static_cast<size_t>(dist.expert[u]) * tiles + p) * tb;
-        cw[i] = __ldcs(reinterpret_cast<const uint2*>(base + 256 * b) + lane);
-        sc[i] = __ldcs(reinterpret_cast<const uint16_t*>(base + 256 * nb + 16 * b) + g);
-      }
-    }
-  };
-  load(warp);
+  const int NS = DN::stages(U);
+  uint8_t* s_stage = smem;
+  uint8_t* s_qh = smem + NS * DN::stage(I);
+  double* s_red = reinterpret_cast<double*>(s_qh + DN::act(I, T * (a.k + a.n_shared)));
+  // the tiles of this CTA and its sequence of (tile, expert) slabs
+  const int ntile = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / G + 1 : 0;
+  const int nslabs = ntile * U;
+  if (tid == 0)
+    for (int q = 0; q < NS && q < nslabs; ++q)
+      dn_issue(a, dist.expert[q % U], blockIdx.x + G * (q / U), s_stage + q * DN::stage(I), &bars[q]);
 
+  MOE_TRACE_POINT(2, 1);
   // ---- after the wait: FP8 re-quantisation of h
   pdl_wait();
+  MOE_TRACE_POINT(2, 2);
   const int nslot = s_nslot;
   if (tid < nslot) {
     const int u = slot_u[tid], tt = slot_t[tid];
@@ -461,54 +516,86 @@ down_combine_kernel(GemvArgs a) {
     if (tid == 0) *a.down_counter = 0;
   }
 
-  // ---- tensor-core GEMV over this warp's (expert, block) pairs
+  MOE_TRACE_POINT(2, 3);
+  // ---- tensor-core GEMV over the slabs; warp w takes blocks w, w+8, ...
+  const int g = lane >> 2, t = lane & 3;
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int q0 = warp; q0 < npairs; q0 += kDNBatch * kDNWarps) {
-    if (q0 != warp) load(q0);
-#pragma unroll
-    for (int i = 0; i < kDNBatch; ++i) {
-      const int q = q0 + i * kDNWarps;
-      if (q < npairs) {
-        const int u = q / nb, b = q % nb;
-        const int slg = g < T ? slot_of[u][g] : -1;
-        uint2 qv = make_uint2(0u, 0u);
-        if (slg >= 0) qv = *reinterpret_cast<const uint2*>(s_qh + static_cast<size_t>(slg) * I + 32 * b + 8 * t);
-        const uint32_t af[4] = {e4m3_lo(cw[i].x), e4m3_lo(cw[i].y), e4m3_hi(cw[i].x), e4m3_hi(cw[i].y)};
-        float d[4];
-        mma_fp8(d, af, qv.x, qv.y);
-        if (2 * t < T) {
-          const double fa = e8m0_to_f64((sc[i] & 0xFFu) + 6), fb = e8m0_to_f64((sc[i] >> 8) + 6);
-          const double c0 = slot_of[u][2 * t] >= 0 ? coef[u][2 * t] : 0.0;
-          acc[0] = fma(static_cast<double>(d[0]), c0 * fa, acc[0]);
-          acc[2] = fma(static_cast<double>(d[2]), c0 * fb, acc[2]);
-          if (2 * t + 1 < T) {
-            const double c1 = slot_of[u][2 * t + 1] >= 0 ? coef[u][2 * t + 1] : 0.0;
-            acc[1] = fma(static_cast<double>(d[1]), c1 * fa, acc[1]);
-            acc[3] = fma(static_cast<double>(d[3]), c1 * fb, acc[3]);
-          }
+  for (int q = 0; q < nslabs; ++q) {
+    const int u = q % U, s = q % NS;
+    const uint8_t* st = s_stage + s * DN::stage(I);
+    if (!mbar_wait_bounded(&bars[s], (q / NS) & 1, a.err)) s_abort = 1;
+    if (*reinterpret_cast<volatile int*>(&s_abort)) break;
+    if (q < 24) MOE_TRACE_POINT(2, 8 + q);
+    const int slg = g < T ? slot_of[u][g] : -1;
+    const double c0 = (2 * t < T && slot_of[u][2 * t] >= 0) ? coef[u][2 * t] : 0.0;
+    const double c1 = (2 * t + 1 < T && slot_of[u][2 * t + 1] >= 0) ? coef[u][2 * t + 1] : 0.0;
+#pragma unroll 3
+    for (int b = warp; b < nb; b += kDNWarps) {
+      const uint2 cw = *reinterpret_cast<const uint2*>(st + 256 * b + 8 * lane);
+      const uint32_t sc = *reinterpret_cast<const uint16_t*>(st + 256 * nb + 16 * b + 2 * g);
+      const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+      uint2 qv = make_uint2(0u, 0u);
+      if (slg >= 0) qv = *reinterpret_cast<const uint2*>(s_qh + static_cast<size_t>(slg) * I + 32 * b + 8 * t);
+      float d[4];
+      mma_fp8(d, af, qv.x, qv.y);
+      if (2 * t < T) {
+        const double fa = e8m0_to_f64((sc & 0xFFu) + 6), fb = e8m0_to_f64((sc >> 8) + 6);
+        acc[0] = fma(static_cast<double>(d[0]), c0 * fa, acc[0]);
+        acc[2] = fma(static_cast<double>(d[2]), c0 * fb, acc[2]);
+        if (2 * t + 1 < T) {
+          acc[1] = fma(static_cast<double>(d[1]), c1 * fa, acc[1]);
+          acc[3] = fma(static_cast<double>(d[3]), c1 * fb, acc[3]);
         }
       }
     }
-  }
-  if (2 * t < T) {
-    s_red[(warp * 16 + g) * T + 2 * t] = acc[0];
-    s_red[(warp * 16 + g + 8) * T + 2 * t] = acc[2];
-    if (2 * t + 1 < T) {
-      s_red[(warp * 16 + g) * T + 2 * t + 1] = acc[1];
-      s_red[(warp * 16 + g + 8) * T + 2 * t + 1] = acc[3];
+    const bool tile_end = u == U - 1;
+    if (NS < nslabs) {
+      __syncthreads();  // stage s fully read
+      if (tid == 0 && q + NS < nslabs)
+        dn_issue(a, dist.expert[(q + NS) % U], blockIdx.x + G * ((q + NS) / U), s_stage + s * DN::stage(I),
+                 &bars[s]);
+    }
+    if (tile_end) {
+      // reduce this tile's rows over the warps and store
+      if (2 * t < T) {
+        s_red[(warp * 16 + g) * T + 2 * t] = acc[0];
+        s_red[(warp * 16 + g + 8) * T + 2 * t] = acc[2];
+        if (2 * t + 1 < T) {
+          s_red[(warp * 16 + g) * T + 2 * t + 1] = acc[1];
+          s_red[(warp * 16 + g + 8) * T + 2 * t + 1] = acc[3];
+        }
+      }
+      acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
+      __syncthreads();
+      const int n0 = 16 * (blockIdx.x + G * (q / U));
+      if (tid < 16 * T) {
+        const int r = tid / T, tt = tid % T;
+        double sum = 0.0;
+        for (int w = 0; w < kDNWarps; ++w) sum += s_red[(w * 16 + r) * T + tt];
+        a.y[static_cast<size_t>(tt) * H + n0 + r] = f64_to_bf16_rne(sum);
+      }
+      __syncthreads();
     }
   }
-  __syncthreads();
-  pdl_trigger();
-  if (tid < 16 * T) {
-    const int r = tid / T, tt = tid % T;
-    double sum = 0.0;
-    for (int w = 0; w < kDNWarps; ++w) sum += s_red[(w * 16 + r) * T + tt];
-    a.y[static_cast<size_t>(tt) * H + n0 + r] = f64_to_bf16_rne(sum);
+  if (__syncthreads_or(s_abort)) {
+    if (tid == 0)
+      for (int s = 0; s < NS; ++s) {
+        mbar_wait_bounded(&bars[s], 0, nullptr);
+        mbar_wait_bounded(&bars[s], 1, nullptr);
+      }
+    return;
   }
+  MOE_TRACE_POINT(2, 4);
+  pdl_trigger();
 }
 
 }  // namespace
+
+#ifdef MOE_TRACE
+extern "C" int moe_trace_read_gemv(unsigned long long* out) {
+  return cudaMemcpyFromSymbol(out, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        void** args) {
@@ -531,22 +618,18 @@ int gemv_chunks_per_cta(int I, int T, int k, int n_shared, int n_ctas) {
 }
 
 size_t gemv_smem_bytes(int H, int I, int T, int k, int n_shared, int n_ctas, int which) {
-  return which == 0 ? GU::total(H, T, gemv_chunks_per_cta(I, T, k, n_shared, n_ctas))
-                    : DN::total(I, T, T * (k + n_shared));
+  const int nmax = gemv_chunks_per_cta(I, T, k, n_shared, n_ctas);
+  return which == 0 ? GU::total(H, T, nmax, GU::stages(H, T, nmax))
+                    : DN::total(I, T, T * k + n_shared, T * (k + n_shared));
 }
 
 cudaError_t launch_gemv(const GemvArgs& a_in, int n_ctas, cudaStream_t stream, Profiler* prof) {
   GemvArgs a = a_in;
   a.gu_nmax = gemv_chunks_per_cta(a.I, a.T, a.k, a.n_shared, n_ctas);
-  const size_t gu_smem = GU::total(a.H, a.T, a.gu_nmax);
-  const size_t dn_smem = DN::total(a.I, a.T, a.T * (a.k + a.n_shared));
-  const int nbw = (a.H / 32 + kGUWarps - 1) / kGUWarps;
-  const void* gu = nbw <= 1 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<1>)
-                   : nbw <= 2 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<2>)
-                   : nbw <= 5 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<5>)
-                   : nbw <= 8 ? reinterpret_cast<const void*>(gateup_swiglu_kernel<8>)
-                              : reinterpret_cast<const void*>(gateup_swiglu_kernel<32>);
-  cudaError_t err = cudaFuncSetAttribute(gu, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  a.gu_stages = GU::stages(a.H, a.T, a.gu_nmax);
+  const size_t gu_smem = GU::total(a.H, a.T, a.gu_nmax, a.gu_stages);
+  const size_t dn_smem = DN::total(a.I, a.T, a.T * a.k + a.n_shared, a.T * (a.k + a.n_shared));
+  cudaError_t err = cudaFuncSetAttribute(gateup_swiglu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(gu_smem));
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -554,11 +637,13 @@ cudaError_t launch_gemv(const GemvArgs& a_in, int n_ctas, cudaStream_t stream, P
   if (err != cudaSuccess) return err;
   void* kargs[] = {&a};
   if (prof) prof->before(1, stream);
-  err = launch_pdl(gu, dim3(n_ctas), dim3(kGUThreads), gu_smem, stream, kargs);
+  err = launch_pdl(reinterpret_cast<const void*>(gateup_swiglu_kernel), dim3(n_ctas), dim3(kGUThreads),
+                   gu_smem, stream, kargs);
   if (prof) prof->after(stream);
   if (err != cudaSuccess) return err;
+  const int tiles = a.H / 16;
   if (prof) prof->before(2, stream);
-  err = launch_pdl(reinterpret_cast<const void*>(down_combine_kernel), dim3(a.H / 16),
+  err = launch_pdl(reinterpret_cast<const void*>(down_combine_kernel), dim3(tiles < n_ctas ? tiles : n_ctas),
                    dim3(kDNThreads), dn_smem, stream, kargs);
   if (prof) prof->after(stream);
   return err;

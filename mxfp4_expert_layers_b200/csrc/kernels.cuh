@@ -48,6 +48,7 @@ struct GemvArgs {
   int* err;             // device error bits
   int prefetch_down;    // gate/up CTAs prefetch the down weights into L2
   int gu_nmax;          // set by launch_gemv: chunks per gate/up CTA at most
+  int gu_stages;        // set by launch_gemv: shared-memory stages per gate/up CTA
   // outputs
   uint16_t* y;          // [T][H]
   moe_debug dbg;

@@ -27,27 +27,26 @@ __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
   return a > b || (a == b && ia < ib);
 }
 
-// Top-k of one token's logits by one warp.  Lane r keeps the r-th selection;
-// the softmax over the selected logits runs on lanes 0..k-1 in float64.
-__device__ void warp_topk(const float* logits, int E, int k, int32_t* ids_out,
-                          float* w_out) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = MOE_MAX_EXPERTS / 32;  // 16 logits per lane
-  float v[kPer];
+// Top-k of one token's logits by the CTA's 4 warps: warp w selects the top-k
+// of experts w*128 .. w*128+127 (4 per lane), then warp 0 merges the 4k
+// candidates (one per lane) and applies the softmax over the selection in
+// float64 on lanes 0..k-1.
+__device__ void cta_topk(const float* logits, int E, int k, int32_t* ids_out, float* w_out,
+                         float* c_val, int* c_id) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float v[4];
   uint32_t taken = 0;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane + 32 * i;
+  for (int i = 0; i < 4; ++i) {
+    const int e = warp * 128 + lane + 32 * i;
     v[i] = e < E ? __ldcg(logits + e) : 0.f;
   }
-  float my_sel = 0.f;
-  int my_id = -1;
   for (int r = 0; r < k; ++r) {
     float bv = 0.f;
     int bi = -1;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
+    for (int i = 0; i < 4; ++i) {
+      const int e = warp * 128 + lane + 32 * i;
       if (e < E && !(taken & (1u << i)) && (bi < 0 || better(v[i], e, bv, bi))) {
         bv = v[i];
         bi = e;
@@ -61,20 +60,46 @@ __device__ void warp_topk(const float* logits, int E, int k, int32_t* ids_out,
         bi = oi;
       }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == r) {
-      my_sel = bv;
-      my_id = bi;
+    if (bi >= 0 && ((bi - warp * 128) & 31) == lane) taken |= 1u << ((bi - warp * 128) >> 5);
+    if (lane == 0) {
+      c_val[warp * MOE_MAX_TOPK + r] = bv;
+      c_id[warp * MOE_MAX_TOPK + r] = bi;
     }
   }
-  // softmax over the selected logits; the first selection is the largest
-  const double top = static_cast<double>(__shfl_sync(0xffffffffu, my_sel, 0));
-  const double z = lane < k ? exp(static_cast<double>(my_sel) - top) : 0.0;
-  const double sum = warp_sum_f64(z);
-  if (lane < k) {
-    ids_out[lane] = my_id;
-    w_out[lane] = static_cast<float>(z / sum);
+  __syncthreads();
+  if (warp == 0) {
+    // lane l holds candidate l (4 warps x up to 8)
+    const bool have = (lane & 7) < k;
+    float cv = have ? c_val[lane] : 0.f;
+    int ci = have ? c_id[lane] : -1;
+    float my_sel = 0.f;
+    int my_id = -1;
+    for (int r = 0; r < k; ++r) {
+      float bv = cv;
+      int bi = ci;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi >= 0 && (bi < 0 || better(ov, oi, bv, bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (ci == bi) ci = -1;  // popped
+      if (lane == r) {
+        my_sel = bv;
+        my_id = bi;
+      }
+    }
+    const double top = static_cast<double>(__shfl_sync(0xffffffffu, my_sel, 0));
+    const double z = lane < k ? exp(static_cast<double>(my_sel) - top) : 0.0;
+    const double sum = warp_sum_f64(z);
+    if (lane < k) {
+      ids_out[lane] = my_id;
+      w_out[lane] = static_cast<float>(z / sum);
+    }
   }
+  __syncthreads();
 }
 
 __device__ __forceinline__ void bf16x2_f32(uint32_t w, float& lo, float& hi) {
@@ -105,6 +130,8 @@ route_kernel(RouteArgs a) {
   constexpr int kRegChunks = NCH;
   __shared__ int s_last;
   __shared__ int s_hist[MOE_MAX_EXPERTS];
+  __shared__ float c_val[kWarps * MOE_MAX_TOPK];
+  __shared__ int c_id[kWarps * MOE_MAX_TOPK];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, H = a.H, T = a.T;
   const int e = blockIdx.x * kWarps + warp;
@@ -112,6 +139,7 @@ route_kernel(RouteArgs a) {
   const int nt = min(kTokTile, T - t0);
   const int nchunk = H / 8;  // 8 bf16 per 16 bytes
 
+  MOE_TRACE_POINT(0, 0);
   // ---- before the wait: router row into registers; shared experts into L2
   uint4 wreg[kRegChunks > 0 ? kRegChunks : 1];
   const uint4* wrow = reinterpret_cast<const uint4*>(a.Wr + static_cast<size_t>(e < E ? e : 0) * H);
@@ -134,8 +162,10 @@ route_kernel(RouteArgs a) {
     }
   }
 
+  MOE_TRACE_POINT(0, 1);
   pdl_wait();
   pdl_trigger();
+  MOE_TRACE_POINT(0, 2);
 
   if (e < E) {
     double acc[kTokTile];
@@ -174,6 +204,7 @@ route_kernel(RouteArgs a) {
     }
   }
 
+  MOE_TRACE_POINT(0, 3);
   // ---- last CTA of this token tile: top-k for its tokens
   __threadfence();
   __syncthreads();
@@ -184,18 +215,24 @@ route_kernel(RouteArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int t = warp; t < nt; t += kWarps)
-    warp_topk(a.logits + static_cast<size_t>(t0 + t) * E, E, a.k,
-              a.ids + static_cast<size_t>(t0 + t) * a.k, a.w + static_cast<size_t>(t0 + t) * a.k);
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    a.tile_counter[blockIdx.y] = 0;
-    const int old = atomicAdd(a.done_counter, 1);
-    s_last = (old == static_cast<int>(gridDim.y) - 1);
+  MOE_TRACE_POINT(0, 4);
+  for (int t = 0; t < nt; ++t)
+    cta_topk(a.logits + static_cast<size_t>(t0 + t) * E, E, a.k, a.ids + static_cast<size_t>(t0 + t) * a.k,
+             a.w + static_cast<size_t>(t0 + t) * a.k, c_val, c_id);
+  MOE_TRACE_POINT(0, 5);
+  if (gridDim.y > 1) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      a.tile_counter[blockIdx.y] = 0;
+      const int old = atomicAdd(a.done_counter, 1);
+      s_last = (old == static_cast<int>(gridDim.y) - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+  } else if (threadIdx.x == 0) {
+    a.tile_counter[0] = 0;
   }
-  __syncthreads();
-  if (!s_last) return;
   // ---- last token tile: counts over all T*k ids
   __threadfence();
   for (int i = threadIdx.x; i < E; i += blockDim.x) s_hist[i] = 0;
@@ -207,10 +244,17 @@ route_kernel(RouteArgs a) {
   __syncthreads();
   if (a.counts)
     for (int i = threadIdx.x; i < E; i += blockDim.x) a.counts[i] = s_hist[i];
-  if (threadIdx.x == 0) *a.done_counter = 0;
+  if (threadIdx.x == 0 && gridDim.y > 1) *a.done_counter = 0;
+  MOE_TRACE_POINT(0, 6);
 }
 
 }  // namespace
+
+#ifdef MOE_TRACE
+extern "C" int moe_trace_read_route(unsigned long long* out) {
+  return cudaMemcpyFromSymbol(out, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   dim3 grid((a.E + kWarps - 1) / kWarps, (a.T + kTokTile - 1) / kTokTile);
