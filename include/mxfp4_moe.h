@@ -144,6 +144,31 @@ int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
                 const float* topk_w, uint16_t* y, const moe_debug* dbg,
                 cudaStream_t stream);
 
+/* moe_forward without a handle and without allocating anything.  The pages
+ * describe no such call; it exists for host code that cannot allocate device
+ * memory -- a serving engine that has given all device memory to its own
+ * pool, or a plugin that may not call cudaMalloc (which can also block the
+ * device) -- and so cannot call moe_create, which allocates a workspace.
+ * The experts run exactly as in moe_forward (same kernels and results), with
+ * their scratch memory (SwiGLU outputs, per-expert amax, a counter: about
+ * 550 KB) in one fixed array inside this library, which every GPU that
+ * loads the library keeps until the process exits.
+ *   - Limits: T in 1..MOE_GEMV_MAX_TOKENS and inter <= 1024; anything larger
+ *     returns MOE_ERR_UNSUPPORTED.  Other arguments as for moe_forward
+ *     (cfg/weights as for moe_create; packed weights), no debug outputs.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing a stream into a graph.
+ *   - Every call on a device shares the one array: calls that overlap on the
+ *     GPU (other streams, other threads) race and give wrong results.  Each
+ *     call clears the parts that must start at zero (cudaMemsetAsync on the
+ *     stream) before its kernels.
+ * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA. */
+int moe_forward_static(const moe_config* cfg, const moe_weights* weights, const uint16_t* x, int T,
+                       const int32_t* topk_ids, const float* topk_w, uint16_t* y,
+                       cudaStream_t stream);
+
 /* Synchronise the stream and report (then clear) device-side errors
  * recorded by earlier calls: MOE_ERR_DEVICE for out-of-range expert ids,
  * MOE_ERR_TIMEOUT if a bounded wait inside a kernel gave up. */

@@ -27,7 +27,7 @@ MOE_GEMV_MAX_TOKENS = 4
 
 EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
-           "moe_profile_begin", "moe_profile_end", "moe_pack_weights")
+           "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static")
 MOE_PROFILE_KERNELS = 4
 KERNEL_NAMES = ("route", "gateup_swiglu", "down_combine", "reserved")
 
@@ -88,6 +88,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_strerror.restype = ctypes.c_char_p
     L.moe_pack_weights.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_mxfp4_weights), i, i,
                                     p, p, p]
+    L.moe_forward_static.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), p, i, p, p, p, p]
     L.moe_profile_begin.argtypes = [p, i]
     L.moe_profile_end.argtypes = [p, p, p]
     L.moe_quantize_fp8.argtypes = [p, i, i, p, p, p]
@@ -164,6 +165,16 @@ def moe_forward(handle: int, x, T: int, topk_ids, topk_w, y, dbg: dict | None = 
         d = ctypes.byref(moe_debug(*[_ptr(dbg.get(f)) for f, _ in moe_debug._fields_]))
     _check(load().moe_forward(handle, _ptr(x), T, _ptr(topk_ids), _ptr(topk_w), _ptr(y), d,
                               _stream(stream)), "moe_forward")
+
+
+def moe_forward_static(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
+                       weights: dict, x, T: int, topk_ids, topk_w, y, stream=None) -> None:
+    """moe_forward for callers that cannot allocate device memory: no handle,
+    scratch in a fixed array of the library (see include/mxfp4_moe.h)."""
+    cfg = moe_config(hidden, inter, n_experts, top_k, n_shared)
+    w = moe_weights(*[_ptr(weights.get(f)) for f, _ in moe_weights._fields_])
+    _check(load().moe_forward_static(ctypes.byref(cfg), ctypes.byref(w), _ptr(x), T, _ptr(topk_ids),
+                                     _ptr(topk_w), _ptr(y), _stream(stream)), "moe_forward_static")
 
 
 def moe_device_error(handle: int, stream=None) -> int:
