@@ -1,11 +1,12 @@
 #!/usr/bin/env python
 """Benchmark of the MXFP4 MoE decode layer on B200.
 
-Default workload (the metric's configuration): one token per step through a
-512-expert layer (top-8 + 1 shared, hidden 2560, width 768, MXFP4 weights,
-FP8 activations), rotating over 64 distinct seeded layers (103 GB) so the
-126 MB L2 never holds a repeated layer.  A step = route + experts + combine
-for one token on one layer.  Prints one JSON line.
+Default workload (the metric's configuration): 512-expert layers (top-8 + 1
+shared, hidden 2560, width 768, MXFP4 weights, FP8 activations), 64 distinct
+seeded layers (103 GB) so the 126 MB L2 never holds a repeated layer.  A step
+= one token through all 64 layers, chained by the residual + RMSNorm harness,
+in one persistent launch (routing, experts and combine of every layer); the
+value is microseconds per token per layer.  Prints one JSON line.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
                   [--workload layer|verify4|stack42]
@@ -38,8 +39,8 @@ METRIC = "MoE-layer decode us/token at B=1 and achieved HBM GB/s (% of B200 peak
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42"])
     p.add_argument("--layers", type=int, default=64)
@@ -151,18 +152,16 @@ class Layers:
 
 
 def alg_bytes(T: int, distinct_routed: int):
-    """Algorithmic bytes of one layer call: weights of the distinct experts
-    touched (routed + shared), the router, activations in/out, and the FP8 h
-    round trip between the two expert kernels."""
+    """Algorithmic bytes of one layer call (one decode launch): weights of the
+    distinct experts touched (routed + shared), the router, x in and y out,
+    and the float32 h written by gate/up and read back for the down step."""
     U = distinct_routed + N_SHARED
     w13 = U * 2 * I * (H // 2 + H // 32)
     w2 = U * H * (I // 2 + I // 32)
     router = E * H * 2
     act = T * H * 2 * 2
-    hbuf = U * T * I * (4 + 1) * 2
-    gateup = w13 + T * H * 2 + U * T * I * 5
-    return {"layer": w13 + w2 + router + act + hbuf, "gateup": gateup, "down": w2 + U * T * I + T * H * 2,
-            "route": router + T * H * 2}
+    hbuf = U * T * I * 4 * 2
+    return {"layer": w13 + w2 + router + act + hbuf, "weights": w13 + w2 + router}
 
 
 # ----------------------------------------------------------- oracle arm --
@@ -219,14 +218,15 @@ def run_reference(args):
 def workload_config(args, layers):
     n = layers.n if layers is not None else args.layers
     if args.workload == "layer":
-        w = f"1-token decode, E=512 top-8 + 1 shared, H=2560, I=768, MXFP4 W4A8, {n} rotating layers"
+        w = (f"1-token decode through {n} distinct E=512 top-8 + 1 shared layers (H=2560, I=768, MXFP4 W4A8), "
+             "chained by the residual + RMSNorm harness, one persistent launch per token")
     elif args.workload == "verify4":
-        w = f"4-token verify call (i.i.d. tokens), E=512 top-8 + 1 shared, {n} rotating layers"
+        w = f"4-token verify call (i.i.d. tokens) through {n} chained E=512 layers, one launch per call"
     else:
-        w = "42-layer decode stack, Zipf(1.1) router bias, residual + RMSNorm chain"
+        w = "42-layer decode stack, Zipf(1.1) router bias, residual + RMSNorm chain, one launch per token"
     c = {"workload": w, "layers_resident": n, "hidden": H, "inter": I, "experts": E, "top_k": K_TOP,
          "shared": N_SHARED,
-         "l2": "inputs larger than L2: distinct layers rotated (" +
+         "l2": "inputs larger than L2: every layer distinct (" +
                f"{n * LAYER_BYTES / 1e9:.1f} GB resident)"}
     if layers is not None and layers.n < layers.requested:
         c["note"] = f"only {layers.n} of {layers.requested} layers fit in free HBM"
@@ -254,34 +254,24 @@ def run_ours(args):
     n_layers = 42 if args.workload == "stack42" else args.layers
     layers = Layers(n_layers, bias=(args.workload == "stack42"), max_tokens=4)
     L = layers.n
+    stack = moe.moe_stack_create(layers.handles)
     stream = torch.cuda.current_stream()
     nsteps = args.warmup + args.steps
 
-    # tokens resident in HBM before timing (fresh draw per step)
+    # fresh tokens per step, resident in HBM before timing
     xs_host = np.stack([synth.hidden_states(0, 1000 + 7919 * rank + i, T, H) for i in range(min(nsteps, 512))])
     xs = torch.from_numpy(xs_host.view(np.int16)).cuda()
-    ids = torch.empty((T, K_TOP), dtype=torch.int32, device="cuda")
-    wts = torch.empty((T, K_TOP), dtype=torch.float32, device="cuda")
-    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
-    # stack: residual + normalised input per layer
     r = torch.empty((T, H), dtype=torch.int16, device="cuda")
-    xin = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    x = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    ids = torch.empty((L, T, K_TOP), dtype=torch.int32, device="cuda")
+    wts = torch.empty((L, T, K_TOP), dtype=torch.float32, device="cuda")
 
-    def step(i):
-        if args.workload == "stack42":
-            x = xs[i % xs.shape[0]]
-            r.copy_(x)
-            xin.copy_(x)
-            for l in range(L):
-                h = layers.handles[l]
-                moe.moe_route(h, xin, T, ids, wts, None, stream)
-                moe.moe_forward(h, xin, T, ids, wts, y, None, stream)
-                moe.moe_residual_rmsnorm(r, y, xin, T, H, 1e-6, stream)
-        else:
-            h = layers.handles[i % L]
-            x = xs[i % xs.shape[0]]
-            moe.moe_route(h, x, T, ids, wts, None, stream)
-            moe.moe_forward(h, x, T, ids, wts, y, None, stream)
+    def step(i, s):
+        # one token (or verify call) through all L layers: one launch
+        x0 = xs[i % xs.shape[0]]
+        r.copy_(x0)
+        x.copy_(x0)
+        moe.moe_stack_decode(stack, r, x, T, 1e-6, ids, wts, None, s)
 
     def barrier():
         torch.cuda.synchronize()
@@ -290,32 +280,19 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     for i in range(args.warmup):
-        step(i)
+        step(i, stream)
     barrier()
+    assert moe.moe_stack_device_error(stack) == moe.MOE_OK
 
-    # ---- headline: CUDA graphs of whole passes over the resident layers
-    per_graph = 1 if args.workload == "stack42" else L
-    full, tail = divmod(args.steps, per_graph)
-    g_full = torch.cuda.CUDAGraph() if full else None
-    g_tail = torch.cuda.CUDAGraph() if tail else None
+    # ---- headline: a CUDA graph of the K steps (one stack launch each)
+    g = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap):
-        stream = cap
-        if g_full is not None:
-            with torch.cuda.graph(g_full, stream=cap):
-                for i in range(per_graph):
-                    step(args.warmup + i)
-        if g_tail is not None:
-            with torch.cuda.graph(g_tail, stream=cap):
-                for i in range(tail):
-                    step(args.warmup + i)
-    stream = torch.cuda.current_stream()
-    for _ in range(2):
-        if g_full is not None:
-            g_full.replay()
-        if g_tail is not None:
-            g_tail.replay()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(args.steps):
+                step(args.warmup + i, cap)
+    g.replay()
     barrier()
     clocks = Clocks(local)
     clocks.start()
@@ -323,90 +300,70 @@ def run_ours(args):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     ev0.record(stream)
-    for _ in range(full):
-        g_full.replay()
-    if g_tail is not None:
-        g_tail.replay()
+    g.replay()
     ev1.record(stream)
     barrier()
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
-
-    # ---- per-kernel times: the same K steps launched eagerly with an event
-    # pair around every kernel (events serialise the kernels)
-    calls_per_handle = args.steps if args.workload == "stack42" else (args.steps + L - 1) // L
-    for h in layers.handles:
-        moe.moe_profile_begin(h, 3 * calls_per_handle + 3)
-    barrier()
-    ev0.record(stream)
-    for i in range(args.warmup, nsteps):
-        step(i)
-    ev1.record(stream)
-    barrier()
-    ms_prof = ev0.elapsed_time(ev1)
-    kern = {}
-    for h in layers.handles:
-        for name, (t, n) in moe.moe_profile_end(h).items():
-            a, b = kern.get(name, (0.0, 0))
-            kern[name] = (a + t, b + n)
-
-    # ---- eager launches without events
-    barrier()
-    ev0.record(stream)
-    for i in range(args.warmup, nsteps):
-        step(i)
-    ev1.record(stream)
-    barrier()
-    ms_eager = ev0.elapsed_time(ev1)
-
+    assert moe.moe_stack_device_error(stack) == moe.MOE_OK
     if world > 1:
         tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
 
-    # distinct experts actually touched (for algorithmic bytes), from the last routing
-    distinct = len(set(ids.cpu().numpy().ravel().tolist()))
-    steps_tokens = args.steps * T
-    per_layer_calls = args.steps * (L if args.workload == "stack42" else 1)
-    if args.workload == "stack42":
-        value = 1e3 * ms / (args.steps * world)          # ms per token of the 42-layer stack -> us
-    else:
-        value = 1e3 * ms / (steps_tokens * world)
-    ab = alg_bytes(T, distinct if T > 1 else K_TOP)
-    layer_us = 1e3 * ms / per_layer_calls
-    gu_ms, gu_n = kern.get("gateup_swiglu", (0.0, 0))
-    dn_ms, dn_n = kern.get("down_combine", (0.0, 0))
-    rt_ms, rt_n = kern.get("route", (0.0, 0))
-    gu_us = 1e3 * gu_ms / max(gu_n, 1)
-    roof = {"bound": "hbm", "kernel": "gateup_swiglu", "achieved": ab["gateup"] / (gu_us * 1e3),
-            "peak": hbm_peak, "unit": "GB/s", "peak_kind": f"{peak_kind} copy bandwidth",
-            "frac": ab["gateup"] / (gu_us * 1e3) / hbm_peak, "traffic": None,
-            "alg_bytes_per_launch": ab["gateup"], "avg_launch_us": gu_us,
-            "other_kernels_us": {"route": 1e3 * rt_ms / max(rt_n, 1), "down_combine": 1e3 * dn_ms / max(dn_n, 1)}}
-    layer_gbs = ab["layer"] / (layer_us * 1e3)
+    # ---- the stack kernel's own duration: events around every launch
+    moe.moe_stack_profile_begin(stack, args.steps + 2)
+    barrier()
+    for i in range(args.warmup, nsteps):
+        step(i, stream)
+    barrier()
+    dk_ms, dk_n = moe.moe_stack_profile_end(stack).get("decode", (0.0, 0))
+    dk_us = 1e3 * dk_ms / max(dk_n, 1)
 
-    # e2e through the public API with pinned host buffers
+    # ---- one launch per layer (moe_decode on each handle), CUDA graph of one pass
+    y1 = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    ids1 = torch.empty((T, K_TOP), dtype=torch.int32, device="cuda")
+    w1 = torch.empty((T, K_TOP), dtype=torch.float32, device="cuda")
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g1, stream=cap):
+            for li in range(L):
+                moe.moe_decode(layers.handles[li], xs[li % xs.shape[0]], T, ids1, w1, y1, None, None, cap)
+    g1.replay()
+    barrier()
+    reps = max(1, min(20, args.steps // 10))
+    ev0.record(stream)
+    for _ in range(reps):
+        g1.replay()
+    ev1.record(stream)
+    barrier()
+    per_call_us = 1e3 * ev0.elapsed_time(ev1) / (reps * L)
+
+    distinct = len(set(ids[-1].cpu().numpy().ravel().tolist()))
+    ab = alg_bytes(T, distinct if T > 1 else K_TOP)
+    layer_us = 1e3 * ms / (args.steps * L)
+    step_us = 1e3 * ms / args.steps
+    if args.workload == "stack42":
+        value = step_us / world                      # us per token through the 42-layer stack
+    else:
+        value = layer_us / (T * world)               # us per token per layer
+    layer_gbs = ab["layer"] / (layer_us * 1e3)
+    roof = {"bound": "hbm", "kernel": "decode_kernel", "achieved": L * ab["layer"] / (dk_us * 1e3),
+            "peak": hbm_peak, "unit": "GB/s", "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+            "frac": L * ab["layer"] / (dk_us * 1e3) / hbm_peak, "traffic": None,
+            "alg_bytes_per_launch": L * ab["layer"], "avg_launch_us": dk_us, "launches_timed": dk_n,
+            "layers_per_launch": L}
+
+    # ---- e2e through the public API with pinned host buffers
     xh = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
-    yh = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    xd = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    xo = torch.empty((T, H), dtype=torch.int16).pin_memory()
     barrier()
     ev0.record(stream)
     for i in range(args.warmup, nsteps):
-        xd.copy_(xh[i % xh.shape[0]], non_blocking=True)
-        if args.workload == "stack42":
-            r.copy_(xd)
-            xin.copy_(xd)
-            for l in range(L):
-                h = layers.handles[l]
-                moe.moe_route(h, xin, T, ids, wts, None, stream)
-                moe.moe_forward(h, xin, T, ids, wts, y, None, stream)
-                moe.moe_residual_rmsnorm(r, y, xin, T, H, 1e-6, stream)
-            yh.copy_(xin, non_blocking=True)
-        else:
-            h = layers.handles[i % L]
-            moe.moe_route(h, xd, T, ids, wts, None, stream)
-            moe.moe_forward(h, xd, T, ids, wts, y, None, stream)
-            yh.copy_(y, non_blocking=True)
+        r.copy_(xh[i % xh.shape[0]], non_blocking=True)
+        x.copy_(r)
+        moe.moe_stack_decode(stack, r, x, T, 1e-6, None, None, None, stream)
+        xo.copy_(x, non_blocking=True)
     ev1.record(stream)
     barrier()
     e2e_ms = ev0.elapsed_time(ev1)
@@ -414,15 +371,16 @@ def run_ours(args):
         tt = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
-    e2e_val = 1e3 * e2e_ms / ((args.steps if args.workload == "stack42" else steps_tokens) * world)
+    e2e_step_us = 1e3 * e2e_ms / args.steps
+    e2e_val = (e2e_step_us if args.workload == "stack42" else e2e_step_us / (L * T)) / world
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = oracle_sample(30, T, budget_s=20.0)
-        cpu = {"value": res["us_per_token"] * (42 if args.workload == "stack42" else 1),
-               "unit": "us/token", "cores": res["cores"], "kind": "oracle", "sample": res["sample"]}
+        cpu = {"value": res["us_per_token"] * (L if args.workload == "stack42" else 1),
+               "unit": "us/token" if args.workload != "stack42" else "us/token (42-layer stack)",
+               "cores": res["cores"], "kind": "oracle", "sample": res["sample"]}
 
-    launches = per_layer_calls * 3 + (args.steps * L if args.workload == "stack42" else 0)
     unit = "us/token" if args.workload != "stack42" else "us/token (42-layer stack)"
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False,
@@ -432,15 +390,21 @@ def run_ours(args):
             "config": workload_config(args, layers),
             "layer_us": layer_us, "layer_gbs": layer_gbs, "layer_frac_of_peak": layer_gbs / hbm_peak,
             "layer_frac_of_8tbs": layer_gbs / 8000.0, "alg_bytes_per_layer": ab["layer"],
+            "per_call_us": per_call_us, "per_call_note": "one moe_decode launch per layer (CUDA graph)",
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": T * H * 2,
                     "d2h_bytes_per_step": T * H * 2},
-            "gpu_launches": launches, "clocks": clk, "timing": "CUDA graphs of whole passes over the layers",
-            "ms_per_step_eager": ms_eager / args.steps, "ms_per_step_eager_with_kernel_events": ms_prof / args.steps}
+            "gpu_launches": args.steps, "clocks": clk,
+            "timing": "CUDA graph of K steps; a step = the token(s) through all resident layers in one launch"}
+    if args.workload == "verify4":
+        line["us_per_call"] = layer_us
+        line["distinct_experts_last_call"] = distinct
     if args.workload == "stack42":
         line["stack_tokens_per_s"] = 1e6 / value
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del g, g1
+    moe.moe_stack_destroy(stack)
     layers.close()
     if world > 1:
         dist.destroy_process_group()

@@ -137,24 +137,41 @@ int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* 
 /* Run the experts of T tokens and combine: x [T][H] bfloat16 (device), the
  * routing from moe_route (or any ids in 0..E-1 and weights the caller
  * chooses), y [T][H] bfloat16 (device, written).  dbg may be NULL.
- * T <= MOE_GEMV_MAX_TOKENS runs the split-K GEMV path; larger T runs the
- * dispatch + grouped-GEMM path.  Ids outside 0..E-1 are skipped and recorded
- * (see moe_device_error).  Errors: MOE_ERR_ARG, MOE_ERR_UNSUPPORTED. */
+ * T <= MOE_GEMV_MAX_TOKENS runs the fused decode kernel (one launch: FP8
+ * quantisation of x, gate/up + SwiGLU, FP8 re-quantisation of h, down and
+ * the weighted combine with the shared experts); larger T runs the dispatch +
+ * grouped-GEMM path.  Ids outside 0..E-1 are skipped and recorded (see
+ * moe_device_error).  Errors: MOE_ERR_ARG, MOE_ERR_UNSUPPORTED. */
 int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
                 const float* topk_w, uint16_t* y, const moe_debug* dbg,
                 cudaStream_t stream);
+
+/* moe_route followed by moe_forward in ONE kernel launch, for decode and
+ * speculative verification (T in 1..MOE_GEMV_MAX_TOKENS): the same ids,
+ * weights, counts and y as the two calls (the routing step of "Ling 3.0 是什么"
+ * on the tanhow.com page -- 8 of 512 routed experts plus the shared one --
+ * followed by the experts).  topk_ids/topk_w [T][top_k] and expert_counts [E]
+ * (may be NULL) are written; the other arguments as for moe_forward.
+ * Requires the whole grid (one CTA per SM) to be resident at once: a launch
+ * that shares the GPU with long-running kernels on other streams waits for
+ * them, and gives up with MOE_ERR_TIMEOUT (moe_device_error) after a second.
+ * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED (T above
+ * MOE_GEMV_MAX_TOKENS or shapes whose tiles do not fit in shared memory). */
+int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
+               int32_t* expert_counts, uint16_t* y, const moe_debug* dbg,
+               cudaStream_t stream);
 
 /* moe_forward without a handle and without allocating anything.  The pages
  * describe no such call; it exists for host code that cannot allocate device
  * memory -- a serving engine that has given all device memory to its own
  * pool, or a plugin that may not call cudaMalloc (which can also block the
  * device) -- and so cannot call moe_create, which allocates a workspace.
- * The experts run exactly as in moe_forward (same kernels and results), with
- * their scratch memory (SwiGLU outputs, per-expert amax, a counter: about
- * 550 KB) in one fixed array inside this library, which every GPU that
- * loads the library keeps until the process exits.
- *   - Limits: T in 1..MOE_GEMV_MAX_TOKENS and inter <= 1024; anything larger
- *     returns MOE_ERR_UNSUPPORTED.  Other arguments as for moe_forward
+ * The experts run exactly as in moe_forward (same kernel and results), with
+ * their scratch memory (SwiGLU outputs, per-expert amax, counters, float64
+ * row accumulators: about 690 KB) in one fixed array inside this library,
+ * which every GPU that loads the library keeps until the process exits.
+ *   - Limits: T in 1..MOE_GEMV_MAX_TOKENS, inter <= 1024 and hidden <= 4096;
+ *     anything larger returns MOE_ERR_UNSUPPORTED.  Other arguments as for moe_forward
  *     (cfg/weights as for moe_create; packed weights), no debug outputs.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
@@ -168,6 +185,46 @@ int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
 int moe_forward_static(const moe_config* cfg, const moe_weights* weights, const uint16_t* x, int T,
                        const int32_t* topk_ids, const float* topk_w, uint16_t* y,
                        cudaStream_t stream);
+
+/* A chained stack of layers run by ONE persistent launch per call (decode
+ * of a whole model's MoE layers for 1..MOE_GEMV_MAX_TOKENS tokens).  The
+ * pages chain MoE layers through the rest of the model, which is not part of
+ * this library; between layers the stack applies the harness step of
+ * moe_residual_rmsnorm (residual add, RMS normalisation without a learned
+ * weight):  for l in 0..L-1:  y = layer_l(x) (routing inside);
+ *   r = bf16(r + y);  x = bf16(r / sqrt(mean(r^2) + eps)).
+ * The next layer's router rows and shared-expert tiles stream into shared
+ * memory while the current layer finishes.
+ *
+ * moe_stack_create: layers[0..n_layers-1] are existing handles with the same
+ * moe_config (their weights are borrowed; the handles must outlive the
+ * stack); allocates the stack's own workspace.  n_layers <= 128.
+ * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE (configs differ), MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA. */
+typedef struct moe_stack_s* moe_stack;
+int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out);
+
+/* Run the stack on T tokens: r [T][H] and x [T][H] bfloat16 (device) hold
+ * the residual and the first layer's input on entry, the final residual and
+ * normalised x on return (in place).  topk_ids/topk_w [L][T][top_k] receive
+ * every layer's routing and x_layers [L][T][H] every layer's input x (each
+ * may be NULL).  Requires the whole grid (one CTA per SM) to be resident at
+ * once, as moe_decode.  Errors: MOE_ERR_ARG (T outside 1..max_tokens of the
+ * layers, at most MOE_GEMV_MAX_TOKENS), MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA; device-side errors via moe_stack_device_error. */
+int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, int32_t* topk_ids,
+                     float* topk_w, uint16_t* x_layers, cudaStream_t stream);
+
+/* As moe_device_error, for a stack. */
+int moe_stack_device_error(moe_stack s, cudaStream_t stream);
+
+/* As moe_profile_begin / moe_profile_end, for a stack (kernel id 1). */
+int moe_stack_profile_begin(moe_stack s, int max_launches);
+int moe_stack_profile_end(moe_stack s, float* ms, int* launches);
+
+/* Free the stack's workspace (synchronises the device first).  NULL is
+ * accepted.  The layer handles are not touched. */
+int moe_stack_destroy(moe_stack s);
 
 /* Synchronise the stream and report (then clear) device-side errors
  * recorded by earlier calls: MOE_ERR_DEVICE for out-of-range expert ids,

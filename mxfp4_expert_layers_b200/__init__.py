@@ -27,9 +27,11 @@ MOE_GEMV_MAX_TOKENS = 4
 
 EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
-           "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static")
+           "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static",
+           "moe_decode", "moe_stack_create", "moe_stack_decode", "moe_stack_device_error",
+           "moe_stack_profile_begin", "moe_stack_profile_end", "moe_stack_destroy")
 MOE_PROFILE_KERNELS = 4
-KERNEL_NAMES = ("route", "gateup_swiglu", "down_combine", "reserved")
+KERNEL_NAMES = ("route", "decode", "grouped_gemm", "reserved")
 
 
 class MoEError(RuntimeError):
@@ -81,9 +83,16 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                              ctypes.POINTER(p)]
     L.moe_route.argtypes = [p, p, i, p, p, p, p]
     L.moe_forward.argtypes = [p, p, i, p, p, p, ctypes.POINTER(moe_debug), p]
+    L.moe_decode.argtypes = [p, p, i, p, p, p, p, ctypes.POINTER(moe_debug), p]
     L.moe_device_error.argtypes = [p, p]
     L.moe_last_path.argtypes = [p]
     L.moe_destroy.argtypes = [p]
+    L.moe_stack_create.argtypes = [p, i, p]
+    L.moe_stack_decode.argtypes = [p, p, p, i, ctypes.c_float, p, p, p, p]
+    L.moe_stack_device_error.argtypes = [p, p]
+    L.moe_stack_profile_begin.argtypes = [p, i]
+    L.moe_stack_profile_end.argtypes = [p, p, p]
+    L.moe_stack_destroy.argtypes = [p]
     L.moe_strerror.argtypes = [i]
     L.moe_strerror.restype = ctypes.c_char_p
     L.moe_pack_weights.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_mxfp4_weights), i, i,
@@ -167,6 +176,17 @@ def moe_forward(handle: int, x, T: int, topk_ids, topk_w, y, dbg: dict | None = 
                               _stream(stream)), "moe_forward")
 
 
+def moe_decode(handle: int, x, T: int, topk_ids, topk_w, y, expert_counts=None,
+               dbg: dict | None = None, stream=None) -> None:
+    """moe_route + moe_forward in one launch (T <= MOE_GEMV_MAX_TOKENS);
+    topk_ids, topk_w and expert_counts are outputs."""
+    d = None
+    if dbg:
+        d = ctypes.byref(moe_debug(*[_ptr(dbg.get(f)) for f, _ in moe_debug._fields_]))
+    _check(load().moe_decode(handle, _ptr(x), T, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts),
+                             _ptr(y), d, _stream(stream)), "moe_decode")
+
+
 def moe_forward_static(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int,
                        weights: dict, x, T: int, topk_ids, topk_w, y, stream=None) -> None:
     """moe_forward for callers that cannot allocate device memory: no handle,
@@ -200,6 +220,39 @@ def moe_profile_end(handle: int) -> dict:
     n = (ctypes.c_int * MOE_PROFILE_KERNELS)()
     _check(load().moe_profile_end(handle, ms, n), "moe_profile_end")
     return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(MOE_PROFILE_KERNELS)}
+
+
+def moe_stack_create(handles) -> int:
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    st = ctypes.c_void_p()
+    _check(load().moe_stack_create(arr, len(handles), ctypes.byref(st)), "moe_stack_create")
+    return st.value
+
+
+def moe_stack_decode(stack: int, r, x, T: int, eps: float = 1e-6, topk_ids=None, topk_w=None,
+                     x_layers=None, stream=None) -> None:
+    """All layers of the stack in one launch; r and x are updated in place."""
+    _check(load().moe_stack_decode(stack, _ptr(r), _ptr(x), T, eps, _ptr(topk_ids), _ptr(topk_w),
+                                   _ptr(x_layers), _stream(stream)), "moe_stack_decode")
+
+
+def moe_stack_device_error(stack: int, stream=None) -> int:
+    return load().moe_stack_device_error(stack, _stream(stream))
+
+
+def moe_stack_profile_begin(stack: int, max_launches: int) -> None:
+    _check(load().moe_stack_profile_begin(stack, max_launches), "moe_stack_profile_begin")
+
+
+def moe_stack_profile_end(stack: int) -> dict:
+    ms = (ctypes.c_float * MOE_PROFILE_KERNELS)()
+    n = (ctypes.c_int * MOE_PROFILE_KERNELS)()
+    _check(load().moe_stack_profile_end(stack, ms, n), "moe_stack_profile_end")
+    return {KERNEL_NAMES[i]: (ms[i], n[i]) for i in range(MOE_PROFILE_KERNELS)}
+
+
+def moe_stack_destroy(stack: int) -> None:
+    _check(load().moe_stack_destroy(stack), "moe_stack_destroy")
 
 
 def moe_quantize_fp8(v, rows: int, cols: int, q, s, stream=None) -> None:

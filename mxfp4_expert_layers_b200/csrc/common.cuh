@@ -66,6 +66,20 @@ __device__ __forceinline__ uint8_t f32_to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
+// d * 2^(E-127+6) as a float64, exactly, for a block sum d of the FP8 MMA
+// (zero or a normal float32: a sum of products of E4M3 codes and E2M1 values
+// scaled by 2^-6 is a multiple of 2^-16) and an E8M0 exponent E, built from
+// the bits with integer operations: the float32 exponent moves into the
+// float64 field with the scale added (bias 1023 - 127 + E - 121), the 23
+// mantissa bits move to the top of the 52.  ebits = (E + 775) << 20.
+__device__ __forceinline__ double scaled_block_f64(float d, uint32_t ebits) {
+  const uint32_t u = __float_as_uint(d);
+  const uint32_t m = u & 0x7FFFFFFFu;
+  const uint32_t hi = m ? ((u & 0x80000000u) | ((m >> 3) + ebits)) : u;
+  return __hiloint2double(static_cast<int>(hi), static_cast<int>(u << 29));
+}
+__device__ __forceinline__ uint32_t block_ebits(uint32_t e8m0) { return (e8m0 + 775u) << 20; }
+
 // E4M3 byte -> half (exact).
 __device__ __forceinline__ __half e4m3_to_half(uint8_t c) {
   __half_raw r = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
@@ -79,39 +93,12 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t byte) {
   return __half2(r);
 }
 
-// float64 -> bfloat16 bits, round to nearest even in one step.  Written out
-// on the bit pattern: keep the top 8 significant bits of the float64 value
-// at the bfloat16 exponent, look at the discarded bits for the rounding.
+// float64 -> bfloat16 bits, round to nearest even in one step (one PTX
+// conversion; the oracle's rounding is the same single rounding).
 __device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
-  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(v));
-  const uint32_t sign = static_cast<uint32_t>(b >> 63) << 15;
-  const int exp = static_cast<int>((b >> 52) & 0x7FF);
-  unsigned long long mant = b & 0xFFFFFFFFFFFFFull;
-  if (exp == 0x7FF) return static_cast<uint16_t>(sign | (mant ? 0x7FC0u : 0x7F80u));
-  if (exp == 0) return static_cast<uint16_t>(sign);          // float64 subnormal -> 0
-  const int e = exp - 1023;                                   // unbiased
-  if (e > 127) return static_cast<uint16_t>(sign | 0x7F80u);  // past the largest: inf
-  // significand with the implicit bit: 53 bits, value = sig * 2^(e-52)
-  unsigned long long sig = mant | (1ull << 52);
-  // bfloat16 keeps 8 significant bits for e >= -126, fewer below (subnormal)
-  int keep_shift = 52 - 7;                                    // bits dropped, normal
-  int be = e + 127;                                           // biased bf16 exponent
-  if (be <= 0) keep_shift += 1 - be;                          // subnormal: drop more
-  if (keep_shift > 63) return static_cast<uint16_t>(sign);
-  unsigned long long q = sig >> keep_shift;
-  const unsigned long long rem = sig & ((1ull << keep_shift) - 1);
-  const unsigned long long half = 1ull << (keep_shift - 1);
-  if (rem > half || (rem == half && (q & 1))) q += 1;
-  uint32_t out;
-  if (be <= 0) {
-    out = static_cast<uint32_t>(q);                           // subnormal (q may reach 0x80)
-  } else {
-    // q in [0x80, 0x100]; 0x100 means the significand rounded up a binade
-    if (q == 0x100) { q = 0x80; be += 1; }
-    if (be >= 0xFF) return static_cast<uint16_t>(sign | 0x7F80u);
-    out = (static_cast<uint32_t>(be) << 7) | static_cast<uint32_t>(q & 0x7F);
-  }
-  return static_cast<uint16_t>(sign | out);
+  uint16_t r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(v));
+  return r;
 }
 
 // ------------------------------------------------------------- reductions --
@@ -167,6 +154,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `ns` nanoseconds inside
+// the instruction while the phase is pending (fewer wasted issue slots).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -180,8 +180,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (long long i = 1; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0 && global_ns() - t0 > kWaitNs) break;
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    if ((i & 15) == 0 && global_ns() - t0 > kWaitNs) break;
   }
   if (err) atomicOr(err, kErrTimeout);
   return false;
@@ -238,6 +238,81 @@ __device__ __forceinline__ uint32_t e2m1x2_bits(uint32_t word, int i) {
 __device__ __forceinline__ uint32_t e4m3x2_bits(uint32_t two) {
   __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
   return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+}
+
+// ------------------------------------------------- FP8 tensor-core GEMV --
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 8 E2M1 codes (one word) -> E4M3 bytes holding value * 2^-6: the codes of
+// the high nibbles (elements 1, 3, 5, 7) and of the low nibbles (0, 2, 4, 6)
+__device__ __forceinline__ uint32_t e4m3_hi(uint32_t w) { return (w & 0x80808080u) | ((w & 0x70707070u) >> 2); }
+__device__ __forceinline__ uint32_t e4m3_lo(uint32_t w) { return e4m3_hi(w << 4); }
+
+// D = A * B (+ C), m16n8k32, A/B e4m3, C/D f32 (mma.sync).  Fragments:
+//   a0 = A[g][4t..4t+3], a1 = A[g+8][4t..], a2 = A[g][16+4t..], a3 = A[g+8][16+4t..]
+//   b0 = B[4t..4t+3][g], b1 = B[16+4t..16+4t+3][g]
+//   d0 = D[g][2t], d1 = D[g][2t+1], d2 = D[g+8][2t], d3 = D[g+8][2t+1]
+__device__ __forceinline__ void mma_fp8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// Position of element k (0..31) of a block inside its permuted activation
+// bytes: group k/8 holds [k0 k2 k4 k6 k1 k3 k5 k7] of that group.
+__device__ __forceinline__ int perm_pos(int k) {
+  const int kk = k & 7;
+  return (k & ~7) + ((kk & 1) ? 4 + (kk >> 1) : (kk >> 1));
+}
+
+// ------------------------------------------- cross-CTA signals (global) --
+// Release/acquire at GPU scope on 32-bit counters in global memory.
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *p >= target, at most kWaitNs of %globaltimer.  Returns false,
+// and records kErrTimeout in *err, if the wait gave up.
+__device__ __forceinline__ bool poll_geq_bounded(const unsigned* p, unsigned target, int* err) {
+  if (ld_acquire_u32(p) >= target) return true;
+  const unsigned long long t0 = global_ns();
+  for (long long i = 1; i < kSpinLimit; ++i) {
+    if (ld_acquire_u32(p) >= target) return true;
+    if ((i & 63) == 0 && global_ns() - t0 > kWaitNs) break;
+  }
+  if (err) atomicOr(err, kErrTimeout);
+  return false;
+}
+
+// ----------------------------------------------------------- router dot --
+__device__ __forceinline__ void bf16x2_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+// acc + the 8 float32 products of two 16-byte chunks of bfloat16 values
+// (each product is exact in float32), summed in float64
+__device__ __forceinline__ double dot8(const uint4 wv, const uint4 xv, double acc) {
+  const uint32_t wp[4] = {wv.x, wv.y, wv.z, wv.w};
+  const uint32_t xp[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float w0, w1, x0, x1;
+    bf16x2_f32(wp[j], w0, w1);
+    bf16x2_f32(xp[j], x0, x1);
+    acc += static_cast<double>(__fmul_rn(w0, x0));
+    acc += static_cast<double>(__fmul_rn(w1, x1));
+  }
+  return acc;
 }
 
 // ------------------------------------------------------------- dispatch --

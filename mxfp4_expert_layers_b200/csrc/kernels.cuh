@@ -33,26 +33,53 @@ struct RouteArgs {
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 int route_tiles(int T);
 
-// GEMV path, T <= MOE_GEMV_MAX_TOKENS (gemv.cu)
-struct GemvArgs {
-  int H, I, E, k, n_shared, T;
-  const uint16_t* x;
-  const int32_t* ids;
-  const float* w;
-  const uint8_t* w13;   // packed gate/up tiles [E+S][I/8][272 H/32]
-  const uint8_t* w2;    // packed down tiles [E+S][H/16][272 I/32]
-  // workspace
-  float* h;             // [kMaxDistinct][kMaxTokGemv][I] SwiGLU output
-  unsigned* amax;       // [kMaxDistinct][kMaxTokGemv] float bits of max|h|, zero between calls
-  int* down_counter;    // zero between calls
-  int* err;             // device error bits
-  int prefetch_down;    // gate/up CTAs prefetch the down weights into L2
-  int gu_nmax;          // set by launch_gemv: chunks per gate/up CTA at most
-  int gu_stages;        // set by launch_gemv: shared-memory stages per gate/up CTA
-  // outputs
-  uint16_t* y;          // [T][H]
-  moe_debug dbg;
+// Fused decode pass, T <= MOE_GEMV_MAX_TOKENS (decode.cu): one persistent
+// launch for one layer or a chained stack of layers (routing optional for a
+// single layer; required for a stack).
+constexpr int kSyncRoute = 0;   // grid arrive/wait counter of the routing step
+constexpr int kSyncExit = 1;    // CTAs finished
+constexpr int kSyncGU = 2;      // CTAs whose gate/up tiles are finished
+constexpr int kSyncY = 3;       // CTAs whose part of y is written
+constexpr int kSyncWords = 64;
+constexpr int kMaxStackLayers = 128;
+struct LayerW {                 // one layer's weights (device pointers)
+  const uint16_t* Wr;           // router [E][H] bf16
+  const float* bias;            // [E] or null
+  const uint8_t* w13;           // packed gate/up tiles
+  const uint8_t* w2;            // packed down tiles
 };
+struct DecodeArgs {
+  int H, I, E, k, n_shared, T;
+  int L;                // layers (1 for moe_decode / moe_forward)
+  int route;            // 1: routing computed inside (ids, w, counts are outputs)
+  LayerW layer0;        // the layer when `layers` is null
+  const LayerW* layers; // [L] device array (stacks)
+  const uint16_t* x;    // [T][H] input of the first layer
+  uint16_t* r_io;       // stack: [T][H] residual in/out (null: plain layer)
+  uint16_t* x_io;       // stack: [T][H] normalised input after the last layer (out)
+  float eps;            // stack: RMS normalisation epsilon
+  int32_t* ids;         // [L][T][k]: input (plain forward), output when routing, or null
+  float* w;             // [L][T][k]
+  int32_t* counts;      // [E] or null (single routed layer)
+  uint16_t* y;          // [T][H] output of a plain layer
+  // workspace; the counters and accumulators are zero between calls
+  float* logits;        // [T][E]
+  float* h;             // [kMaxDistinct][kMaxTokGemv][I]
+  unsigned* amax;       // [L][kMaxDistinct][kMaxTokGemv]
+  unsigned* sync;       // [kSyncWords]
+  unsigned* tile_cnt;   // [H/16]
+  double* yacc;         // [kMaxTokGemv][H]
+  uint16_t* ybuf;       // [2][T][H] y of stacked layers
+  int* err;
+  moe_debug dbg;        // plain layer only
+  uint16_t* dbg_x;      // [L][T][H] input x of every layer, or null
+  // shared-memory plan (decode_plan)
+  int ng_slots, nd_slots;  // gate/up and down ring slots
+  int dn_off, rr_off, xq_off, red_off, qh_off, yrow_off, rs_off, yrow_len, smem_bytes;
+};
+bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget);
+cudaError_t launch_decode(const DecodeArgs& a, int n_ctas, cudaStream_t stream);
+int decode_static_smem();
 
 // Optional per-kernel event timing (owned by the handle).
 struct Profiler {
@@ -67,8 +94,6 @@ struct Profiler {
   }
 };
 
-size_t gemv_smem_bytes(int H, int I, int T, int k, int n_shared, int n_ctas, int which);
-int gemv_chunks_per_cta(int I, int T, int k, int n_shared, int n_ctas);
 
 // Weight packing (pack.cu)
 struct PackArgs {
@@ -82,7 +107,6 @@ struct PackArgs {
   uint8_t* w2_out;
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t stream);
-cudaError_t launch_gemv(const GemvArgs& a, int n_ctas, cudaStream_t stream, Profiler* prof);
 
 // Per-row FP8 quantisation (quant.cu)
 cudaError_t launch_quantize_rows(const float* v, int rows, int cols, uint8_t* q, float* s,

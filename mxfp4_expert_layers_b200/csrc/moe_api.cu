@@ -20,9 +20,12 @@ struct moe_handle_s {
   int* done_counter;   // [1]
   int* err;            // [1]
   unsigned* amax;      // [kMaxDistinct][kMaxTokGemv]
-  int* down_counter;   // [1]
   float* h;            // [kMaxDistinct][kMaxTokGemv][I]
+  unsigned* sync;      // [kSyncWords]
+  unsigned* tile_cnt;  // [H/16]
+  double* yacc;        // [kMaxTokGemv][H]
   int n_sms;
+  int smem_budget;     // dynamic shared memory available to the decode kernel
   moe::Profiler prof;
   bool profiling;
 };
@@ -83,16 +86,23 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const int E = cfg->n_experts, I = cfg->inter;
   const size_t n_logits = up256(static_cast<size_t>(max_tokens) * E * 4);
   const size_t n_tiles = up256(static_cast<size_t>(moe::route_tiles(max_tokens)) * 4);
-  const size_t n_small = 256;  // done_counter, err, down_counter
+  const size_t n_small = 256;  // done_counter, err
   const size_t n_amax = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * I * 4);
-  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h;
-  int dev = 0;
+  const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
+  const size_t n_tcnt = up256(static_cast<size_t>(cfg->hidden / 16) * 4);
+  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * cfg->hidden * 8);
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tcnt + n_yacc;
+  int dev = 0, optin = 0;
+  const int static_smem = moe::decode_static_smem();
   if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+      static_smem < 0) {
     delete h;
     return MOE_ERR_CUDA;
   }
+  h->smem_budget = optin - static_smem - 256;
   if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
     delete h;
     return MOE_ERR_CUDA;
@@ -107,9 +117,12 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->tile_counter = reinterpret_cast<int*>(p); p += n_tiles;
   h->done_counter = reinterpret_cast<int*>(p);
   h->err = reinterpret_cast<int*>(p + 64);
-  h->down_counter = reinterpret_cast<int*>(p + 128); p += n_small;
+  p += n_small;
   h->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
-  h->h = reinterpret_cast<float*>(p);
+  h->h = reinterpret_cast<float*>(p); p += n_h;
+  h->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
+  h->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
+  h->yacc = reinterpret_cast<double*>(p);
   *out = h;
   return MOE_OK;
 }
@@ -135,23 +148,53 @@ int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* 
   return cuda_err(e);
 }
 
+namespace {
+
+// The fused decode launch shared by moe_forward (ids given) and moe_decode
+// (routing inside).
+int decode_call(moe_handle h, const uint16_t* x, int T, int route, int32_t* ids, float* w, int32_t* counts,
+                uint16_t* y, const moe_debug* dbg, cudaStream_t stream) {
+  const moe_config& c = h->cfg;
+  moe::DecodeArgs a{};
+  a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
+  a.L = 1;
+  a.route = route;
+  a.layer0 = moe::LayerW{h->w.router_w, h->w.router_bias, h->w.w13, h->w.w2};
+  a.x = x;
+  a.ids = ids; a.w = w; a.counts = counts;
+  a.logits = h->logits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.tile_cnt = h->tile_cnt;
+  a.yacc = h->yacc; a.err = h->err;
+  a.y = y;
+  if (dbg) a.dbg = *dbg;
+  if (!moe::decode_plan(a, h->n_sms, h->smem_budget)) return MOE_ERR_UNSUPPORTED;
+  h->last_path = 1;
+  if (h->profiling) h->prof.before(1, stream);
+  const cudaError_t e = moe::launch_decode(a, h->n_sms, stream);
+  if (h->profiling) h->prof.after(stream);
+  return cuda_err(e);
+}
+
+}  // namespace
+
 int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
                 const float* topk_w, uint16_t* y, const moe_debug* dbg, cudaStream_t stream) {
   if (!h || !x || !topk_ids || !topk_w || !y) return MOE_ERR_ARG;
   if (T < 1 || T > h->max_tokens) return MOE_ERR_ARG;
   if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y)) return MOE_ERR_ALIGN;
-  const moe_config& c = h->cfg;
   if (T > MOE_GEMV_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
-  moe::GemvArgs a{};
-  a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
-  a.x = x; a.ids = topk_ids; a.w = topk_w;
-  a.w13 = h->w.w13; a.w2 = h->w.w2;
-  a.h = h->h; a.amax = h->amax; a.down_counter = h->down_counter; a.err = h->err;
-  a.prefetch_down = 1;
-  a.y = y;
-  if (dbg) a.dbg = *dbg;
-  h->last_path = 1;
-  return cuda_err(moe::launch_gemv(a, h->n_sms, stream, h->profiling ? &h->prof : nullptr));
+  return decode_call(h, x, T, 0, const_cast<int32_t*>(topk_ids), const_cast<float*>(topk_w), nullptr, y, dbg,
+                     stream);
+}
+
+int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
+               int32_t* expert_counts, uint16_t* y, const moe_debug* dbg, cudaStream_t stream) {
+  if (!h || !x || !topk_ids || !topk_w || !y) return MOE_ERR_ARG;
+  if (T < 1 || T > h->max_tokens) return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y) ||
+      (expert_counts && !aligned4(expert_counts)))
+    return MOE_ERR_ALIGN;
+  if (T > MOE_GEMV_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+  return decode_call(h, x, T, 1, topk_ids, topk_w, expert_counts, y, dbg, stream);
 }
 
 int moe_device_error(moe_handle h, cudaStream_t stream) {
@@ -159,7 +202,16 @@ int moe_device_error(moe_handle h, cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
   int e = 0;
   if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
-  if (e && cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (e) {
+    // a kernel that gave up may have left its counters and accumulators set
+    if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(h->amax, 0, static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4) != cudaSuccess ||
+        cudaMemset(h->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
+        cudaMemset(h->tile_cnt, 0, static_cast<size_t>(h->cfg.hidden / 16) * 4) != cudaSuccess ||
+        cudaMemset(h->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.hidden * 8) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (e & moe::kErrTimeout) return MOE_ERR_TIMEOUT;
   if (e & moe::kErrBadId) return MOE_ERR_DEVICE;
   return MOE_OK;
@@ -250,6 +302,188 @@ int moe_residual_rmsnorm(uint16_t* r, const uint16_t* y, uint16_t* x_next, int T
                          cudaStream_t stream) {
   if (!r || !y || !x_next || T < 1 || H < 1 || !(eps >= 0.f)) return MOE_ERR_ARG;
   return cuda_err(moe::launch_residual_rmsnorm(r, y, x_next, T, H, eps, stream));
+}
+
+// ------------------------------------------------------------------ stack --
+
+struct moe_stack_s {
+  moe_config cfg;
+  int L;
+  int max_tokens;
+  void* ws;
+  moe::LayerW* layers;   // [L] device
+  float* logits;
+  float* h;
+  unsigned* amax;        // [L][kMaxDistinct][kMaxTokGemv]
+  unsigned* sync;
+  unsigned* tile_cnt;
+  double* yacc;
+  uint16_t* ybuf;        // [2][kMaxTokGemv][H]
+  int* err;
+  int n_sms;
+  int smem_budget;
+  moe::Profiler prof;
+  bool profiling;
+};
+
+int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
+  if (!layers || !out || n_layers < 1) return MOE_ERR_ARG;
+  if (n_layers > moe::kMaxStackLayers) return MOE_ERR_UNSUPPORTED;
+  for (int l = 0; l < n_layers; ++l)
+    if (!layers[l]) return MOE_ERR_ARG;
+  const moe_config c = layers[0]->cfg;
+  int max_tokens = MOE_GEMV_MAX_TOKENS;
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_config& d = layers[l]->cfg;
+    if (d.hidden != c.hidden || d.inter != c.inter || d.n_experts != c.n_experts || d.top_k != c.top_k ||
+        d.n_shared != c.n_shared)
+      return MOE_ERR_SHAPE;
+    if (layers[l]->max_tokens < max_tokens) max_tokens = layers[l]->max_tokens;
+  }
+  moe_stack s = new (std::nothrow) moe_stack_s();
+  if (!s) return MOE_ERR_CUDA;
+  s->cfg = c;
+  s->L = n_layers;
+  s->max_tokens = max_tokens;
+  s->n_sms = layers[0]->n_sms;
+  s->smem_budget = layers[0]->smem_budget;
+  const size_t n_layers_b = up256(static_cast<size_t>(n_layers) * sizeof(moe::LayerW));
+  const size_t n_logits = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.n_experts * 4);
+  const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * c.inter * 4);
+  const size_t n_amax = up256(static_cast<size_t>(n_layers) * moe::kMaxDistinct * moe::kMaxTokGemv * 4);
+  const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
+  const size_t n_tcnt = up256(static_cast<size_t>(c.hidden / 16) * 4);
+  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.hidden * 8);
+  const size_t n_ybuf = up256(static_cast<size_t>(2) * moe::kMaxTokGemv * c.hidden * 2);
+  const size_t n_err = 256;
+  const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_tcnt + n_yacc + n_ybuf + n_err;
+  if (cudaMalloc(&s->ws, bytes) != cudaSuccess) {
+    delete s;
+    return MOE_ERR_CUDA;
+  }
+  uint8_t* p = static_cast<uint8_t*>(s->ws);
+  s->layers = reinterpret_cast<moe::LayerW*>(p); p += n_layers_b;
+  s->logits = reinterpret_cast<float*>(p); p += n_logits;
+  s->h = reinterpret_cast<float*>(p); p += n_h;
+  s->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
+  s->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
+  s->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
+  s->yacc = reinterpret_cast<double*>(p); p += n_yacc;
+  s->ybuf = reinterpret_cast<uint16_t*>(p); p += n_ybuf;
+  s->err = reinterpret_cast<int*>(p);
+  moe::LayerW* host = new (std::nothrow) moe::LayerW[n_layers];
+  if (!host) {
+    cudaFree(s->ws);
+    delete s;
+    return MOE_ERR_CUDA;
+  }
+  for (int l = 0; l < n_layers; ++l)
+    host[l] = moe::LayerW{layers[l]->w.router_w, layers[l]->w.router_bias, layers[l]->w.w13, layers[l]->w.w2};
+  const bool okc = cudaMemset(s->ws, 0, bytes) == cudaSuccess &&
+                   cudaMemcpy(s->layers, host, static_cast<size_t>(n_layers) * sizeof(moe::LayerW),
+                              cudaMemcpyHostToDevice) == cudaSuccess &&
+                   cudaDeviceSynchronize() == cudaSuccess;
+  delete[] host;
+  if (!okc) {
+    cudaFree(s->ws);
+    delete s;
+    return MOE_ERR_CUDA;
+  }
+  *out = s;
+  return MOE_OK;
+}
+
+int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, int32_t* topk_ids,
+                     float* topk_w, uint16_t* x_layers, cudaStream_t stream) {
+  if (!s || !r || !x) return MOE_ERR_ARG;
+  if (T < 1 || T > s->max_tokens || !(eps >= 0.f)) return MOE_ERR_ARG;
+  if (!aligned16(r) || !aligned16(x) || (topk_ids && !aligned4(topk_ids)) || (topk_w && !aligned4(topk_w)) ||
+      (x_layers && !aligned16(x_layers)))
+    return MOE_ERR_ALIGN;
+  const moe_config& c = s->cfg;
+  moe::DecodeArgs a{};
+  a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
+  a.L = s->L;
+  a.route = 1;
+  a.layers = s->layers;
+  a.x = x; a.r_io = r; a.x_io = x; a.eps = eps;
+  a.ids = topk_ids; a.w = topk_w;
+  a.logits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync; a.tile_cnt = s->tile_cnt;
+  a.yacc = s->yacc; a.ybuf = s->ybuf; a.err = s->err;
+  a.dbg_x = x_layers;
+  if (!moe::decode_plan(a, s->n_sms, s->smem_budget)) return MOE_ERR_UNSUPPORTED;
+  if (s->profiling) s->prof.before(1, stream);
+  const cudaError_t e = moe::launch_decode(a, s->n_sms, stream);
+  if (s->profiling) s->prof.after(stream);
+  return cuda_err(e);
+}
+
+int moe_stack_device_error(moe_stack s, cudaStream_t stream) {
+  if (!s) return MOE_ERR_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int e = 0;
+  if (cudaMemcpy(&e, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (e) {
+    if (cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(s->amax, 0, static_cast<size_t>(s->L) * moe::kMaxDistinct * moe::kMaxTokGemv * 4) != cudaSuccess ||
+        cudaMemset(s->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
+        cudaMemset(s->tile_cnt, 0, static_cast<size_t>(s->cfg.hidden / 16) * 4) != cudaSuccess ||
+        cudaMemset(s->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.hidden * 8) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (e & moe::kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (e & moe::kErrBadId) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+int moe_stack_profile_begin(moe_stack s, int max_launches) {
+  if (!s || max_launches < 1 || max_launches > (1 << 20)) return MOE_ERR_ARG;
+  free_profiler(s->prof);
+  s->prof.ev = new (std::nothrow) cudaEvent_t[2 * max_launches];
+  s->prof.kid = new (std::nothrow) int[max_launches];
+  if (!s->prof.ev || !s->prof.kid) { free_profiler(s->prof); return MOE_ERR_CUDA; }
+  for (int i = 0; i < 2 * max_launches; ++i) {
+    if (cudaEventCreate(&s->prof.ev[i]) != cudaSuccess) {
+      s->prof.cap = i / 2;
+      free_profiler(s->prof);
+      return MOE_ERR_CUDA;
+    }
+    s->prof.cap = (i + 1) / 2;
+  }
+  s->prof.cap = max_launches;
+  s->prof.n = 0;
+  s->profiling = true;
+  return MOE_OK;
+}
+
+int moe_stack_profile_end(moe_stack s, float* ms, int* launches) {
+  if (!s || !ms || !launches) return MOE_ERR_ARG;
+  s->profiling = false;
+  for (int k = 0; k < MOE_PROFILE_KERNELS; ++k) { ms[k] = 0.f; launches[k] = 0; }
+  int rc = MOE_OK;
+  for (int i = 0; i < s->prof.n; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(s->prof.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, s->prof.ev[2 * i], s->prof.ev[2 * i + 1]) != cudaSuccess) {
+      rc = MOE_ERR_CUDA;
+      continue;
+    }
+    ms[s->prof.kid[i]] += t;
+    launches[s->prof.kid[i]] += 1;
+  }
+  free_profiler(s->prof);
+  return rc;
+}
+
+int moe_stack_destroy(moe_stack s) {
+  if (!s) return MOE_OK;
+  int rc = MOE_OK;
+  free_profiler(s->prof);
+  if (cudaDeviceSynchronize() != cudaSuccess) rc = MOE_ERR_CUDA;
+  if (s->ws && cudaFree(s->ws) != cudaSuccess) rc = MOE_ERR_CUDA;
+  delete s;
+  return rc;
 }
 
 }  // extern "C"

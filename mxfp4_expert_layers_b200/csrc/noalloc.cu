@@ -1,4 +1,4 @@
-// moe_forward_static: the expert kernels of moe_forward with their scratch
+// moe_forward_static: the expert kernel of moe_forward with its scratch
 // memory in a fixed array of this library instead of a handle's workspace,
 // for host code that must not allocate device memory.
 //
@@ -18,13 +18,22 @@ namespace moe {
 namespace {
 
 constexpr int kStaticMaxInter = 1024;
+constexpr int kStaticMaxHidden = 4096;
 constexpr size_t kStaticH = static_cast<size_t>(kMaxDistinct) * kMaxTokGemv * kStaticMaxInter * sizeof(float);
-constexpr size_t kStaticAmax = static_cast<size_t>(kMaxDistinct) * kMaxTokGemv * sizeof(unsigned);
-// layout: h | amax | down counter | error word (the last three start at zero)
+constexpr size_t kStaticAmax = 1024;     // >= kMaxDistinct * kMaxTokGemv unsigned
+constexpr size_t kStaticSync = 256;      // >= kSyncWords unsigned
+constexpr size_t kStaticTile = (kStaticMaxHidden / 16) * sizeof(unsigned);
+constexpr size_t kStaticYacc = static_cast<size_t>(kMaxTokGemv) * kStaticMaxHidden * sizeof(double);
+static_assert(kStaticAmax >= kMaxDistinct * kMaxTokGemv * sizeof(unsigned), "amax area");
+static_assert(kStaticSync >= kSyncWords * sizeof(unsigned), "counter area");
+// layout: h | amax | counters | row-tile counters | float64 accumulators | error
+// word (everything after h starts at zero)
 constexpr size_t kOffAmax = kStaticH;
-constexpr size_t kOffCounter = kOffAmax + kStaticAmax;
-constexpr size_t kOffErr = kOffCounter + 64;
-constexpr size_t kStaticBytes = kOffErr + 64;
+constexpr size_t kOffSync = kOffAmax + kStaticAmax;
+constexpr size_t kOffTile = kOffSync + kStaticSync;
+constexpr size_t kOffYacc = kOffTile + kStaticTile;
+constexpr size_t kOffErr = kOffYacc + kStaticYacc;
+constexpr size_t kStaticBytes = kOffErr + 256;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 
@@ -32,9 +41,10 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 unsigned char* g_addr[kMaxDevices];
 int g_sms[kMaxDevices];
+int g_budget[kMaxDevices];
 
 // Device address of the scratch array on the current device (looked up once).
-int scratch_for_current_device(unsigned char** addr, int* n_sms) {
+int scratch_for_current_device(unsigned char** addr, int* n_sms, int* budget) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
@@ -42,13 +52,19 @@ int scratch_for_current_device(unsigned char** addr, int* n_sms) {
   if (!g_addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    int sms = 0, optin = 0;
+    const int static_smem = decode_static_smem();
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        static_smem < 0)
+      return MOE_ERR_CUDA;
     g_addr[dev] = static_cast<unsigned char*>(p);
     g_sms[dev] = sms;
+    g_budget[dev] = optin - static_smem - 256;
   }
   *addr = g_addr[dev];
   *n_sms = g_sms[dev];
+  *budget = g_budget[dev];
   return MOE_OK;
 }
 
@@ -69,25 +85,32 @@ extern "C" int moe_forward_static(const moe_config* cfg, const moe_weights* w, c
       cfg->top_k > MOE_MAX_TOPK || cfg->top_k > cfg->n_experts || cfg->n_shared < 0 ||
       cfg->n_shared > MOE_MAX_SHARED)
     return MOE_ERR_SHAPE;
-  if (T < 1 || T > MOE_GEMV_MAX_TOKENS || cfg->inter > kStaticMaxInter) return MOE_ERR_UNSUPPORTED;
+  if (T < 1 || T > MOE_GEMV_MAX_TOKENS || cfg->inter > kStaticMaxInter || cfg->hidden > kStaticMaxHidden)
+    return MOE_ERR_UNSUPPORTED;
   if (!al16(x) || !al16(w->w13) || !al16(w->w2) || !al4(topk_ids) || !al4(topk_w) || !al4(y))
     return MOE_ERR_ALIGN;
   unsigned char* base = nullptr;
-  int sms = 0;
-  const int rc = scratch_for_current_device(&base, &sms);
+  int sms = 0, budget = 0;
+  const int rc = scratch_for_current_device(&base, &sms, &budget);
   if (rc != MOE_OK) return rc;
-  // the parts that must start at zero: amax, the down counter, the error word
-  if (cudaMemsetAsync(base + kOffAmax, 0, kStaticBytes - kOffAmax, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  GemvArgs a{};
+  DecodeArgs a{};
   a.H = cfg->hidden; a.I = cfg->inter; a.E = cfg->n_experts; a.k = cfg->top_k; a.n_shared = cfg->n_shared;
   a.T = T;
-  a.x = x; a.ids = topk_ids; a.w = topk_w;
-  a.w13 = w->w13; a.w2 = w->w2;
+  a.L = 1;
+  a.route = 0;
+  a.layer0 = LayerW{nullptr, nullptr, w->w13, w->w2};
+  a.x = x;
+  a.ids = const_cast<int32_t*>(topk_ids);
+  a.w = const_cast<float*>(topk_w);
   a.h = reinterpret_cast<float*>(base);
   a.amax = reinterpret_cast<unsigned*>(base + kOffAmax);
-  a.down_counter = reinterpret_cast<int*>(base + kOffCounter);
+  a.sync = reinterpret_cast<unsigned*>(base + kOffSync);
+  a.tile_cnt = reinterpret_cast<unsigned*>(base + kOffTile);
+  a.yacc = reinterpret_cast<double*>(base + kOffYacc);
   a.err = reinterpret_cast<int*>(base + kOffErr);
-  a.prefetch_down = 1;
   a.y = y;
-  return launch_gemv(a, sms, stream, nullptr) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (!decode_plan(a, sms, budget)) return MOE_ERR_UNSUPPORTED;
+  // the parts that must start at zero
+  if (cudaMemsetAsync(base + kOffAmax, 0, kStaticBytes - kOffAmax, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_decode(a, sms, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

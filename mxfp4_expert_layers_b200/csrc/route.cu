@@ -102,26 +102,6 @@ __device__ void cta_topk(const float* logits, int E, int k, int32_t* ids_out, fl
   __syncthreads();
 }
 
-__device__ __forceinline__ void bf16x2_f32(uint32_t w, float& lo, float& hi) {
-  lo = __uint_as_float(w << 16);
-  hi = __uint_as_float(w & 0xFFFF0000u);
-}
-
-// acc += sum of the 8 exact float32 products of two 16-byte chunks
-__device__ __forceinline__ double dot8(const uint4 wv, const uint4 xv, double acc) {
-  const uint32_t wp[4] = {wv.x, wv.y, wv.z, wv.w};
-  const uint32_t xp[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    float w0, w1, x0, x1;
-    bf16x2_f32(wp[j], w0, w1);
-    bf16x2_f32(xp[j], x0, x1);
-    acc += static_cast<double>(__fmul_rn(w0, x0));
-    acc += static_cast<double>(__fmul_rn(w1, x1));
-  }
-  return acc;
-}
-
 // NCH = 16-byte chunks of a router row per lane kept in registers (0: rows
 // longer than 16 chunks per lane, streamed from global memory instead).
 template <int NCH>

@@ -100,18 +100,29 @@ class GpuLayer:
         moe.moe_route(self.handle, x_dev, T, ids, w, counts, torch.cuda.current_stream())
         return ids, w, counts
 
-    def forward(self, x_dev, T, ids, w, debug=True):
+    def _debug_buffers(self, T):
         S = self.k + self.S
+        return {"xq": torch.empty((T, self.H), dtype=torch.uint8, device="cuda"),
+                "xs": torch.empty((T,), dtype=torch.float32, device="cuda"),
+                "h": torch.empty((T, S, self.I), dtype=torch.float32, device="cuda"),
+                "qh": torch.empty((T, S, self.I), dtype=torch.uint8, device="cuda"),
+                "sh": torch.empty((T, S), dtype=torch.float32, device="cuda")}
+
+    def forward(self, x_dev, T, ids, w, debug=True):
         y = torch.empty((T, self.H), dtype=torch.int16, device="cuda")
-        dbg = None
-        if debug:
-            dbg = {"xq": torch.empty((T, self.H), dtype=torch.uint8, device="cuda"),
-                   "xs": torch.empty((T,), dtype=torch.float32, device="cuda"),
-                   "h": torch.empty((T, S, self.I), dtype=torch.float32, device="cuda"),
-                   "qh": torch.empty((T, S, self.I), dtype=torch.uint8, device="cuda"),
-                   "sh": torch.empty((T, S), dtype=torch.float32, device="cuda")}
+        dbg = self._debug_buffers(T) if debug else None
         moe.moe_forward(self.handle, x_dev, T, ids, w, y, dbg, torch.cuda.current_stream())
         return y, dbg
+
+    def decode(self, x_dev, T, debug=True):
+        """moe_decode: routing and experts in one launch."""
+        ids = torch.empty((T, self.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, self.k), dtype=torch.float32, device="cuda")
+        counts = torch.empty((self.E,), dtype=torch.int32, device="cuda")
+        y = torch.empty((T, self.H), dtype=torch.int16, device="cuda")
+        dbg = self._debug_buffers(T) if debug else None
+        moe.moe_decode(self.handle, x_dev, T, ids, w, y, counts, dbg, torch.cuda.current_stream())
+        return ids, w, counts, y, dbg
 
 
 def check_route(g_ids, g_w, g_counts, ref):

@@ -26,14 +26,21 @@ def _oracle(layer: GpuLayer, x_bits):
     return OM.moe_layer(x_bits, layer.host, layer.E, layer.k, layer.I, layer.S)
 
 
-def _run(layer: GpuLayer, x_bits, debug=True):
+def _run(layer: GpuLayer, x_bits, debug=True, mode="split"):
+    """mode "split": moe_route then moe_forward; "fused": moe_decode."""
     T = x_bits.shape[0]
     xd = to_dev_u16(x_bits)
-    ids, w, counts = layer.route(xd, T)
-    y, dbg = layer.forward(xd, T, ids, w, debug)
+    if mode == "split":
+        ids, w, counts = layer.route(xd, T)
+        y, dbg = layer.forward(xd, T, ids, w, debug)
+    else:
+        ids, w, counts, y, dbg = layer.decode(xd, T, debug)
     torch.cuda.synchronize()
     assert moe.moe_device_error(layer.handle) == moe.MOE_OK
     return ids, w, counts, y, dbg
+
+
+MODES = ["split", "fused"]
 
 
 # ------------------------------------------------------------ generators --
@@ -174,15 +181,16 @@ def test_gpu_route_ties_go_to_lower_index():
 
 # ------------------------------------------------------------- forward --
 
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("n_shared", [0, 1, 2])
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
-def test_gpu_forward_small_shapes(T, n_shared):
+def test_gpu_forward_small_shapes(T, n_shared, mode):
     E, H, I, k = 8, 128, 64, 2
     L = GpuLayer(2, T, E, H, I, k=k, n_shared=n_shared, fill="host")
     try:
         for step in range(3):
             x = synth.hidden_states(2, 10 * T + step, T, H)
-            ids, w, counts, y, dbg = _run(L, x)
+            ids, w, counts, y, dbg = _run(L, x, mode=mode)
             ref = _oracle(L, x)
             check_route(ids, w, counts, ref)
             check_forward(y, dbg, ref)
@@ -190,13 +198,14 @@ def test_gpu_forward_small_shapes(T, n_shared):
         L.close()
 
 
-def test_gpu_forward_config0_single_token():
+@pytest.mark.parametrize("mode", MODES)
+def test_gpu_forward_config0_single_token(mode):
     """One token, E = 32 routed top-8 + 1 shared, H 2560, I 768, seed 0."""
     L = GpuLayer(0, 0, 32)
     try:
         for step in range(4):
             x = synth.hidden_states(0, step, 1, H0)
-            ids, w, counts, y, dbg = _run(L, x)
+            ids, w, counts, y, dbg = _run(L, x, mode=mode)
             ref = _oracle(L, x)
             check_route(ids, w, counts, ref)
             st = check_forward(y, dbg, ref)
@@ -205,14 +214,15 @@ def test_gpu_forward_config0_single_token():
         L.close()
 
 
-def test_gpu_forward_config1_full_layer():
+@pytest.mark.parametrize("mode", MODES)
+def test_gpu_forward_config1_full_layer(mode):
     """E = 512 (the 1.6 GB layer) at full size; tokens one at a time."""
     for layer in (0, 1):
         L = GpuLayer(0, layer, 512)
         try:
             for step in range(3):
                 x = synth.hidden_states(0, 1000 + 10 * layer + step, 1, H0)
-                ids, w, counts, y, dbg = _run(L, x)
+                ids, w, counts, y, dbg = _run(L, x, mode=mode)
                 ref = _oracle(L, x)
                 check_route(ids, w, counts, ref)
                 check_forward(y, dbg, ref)
@@ -227,8 +237,9 @@ def test_gpu_forward_config1_full_layer():
             L.close()
 
 
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("kind", ["iid", "clustered"])
-def test_gpu_forward_config2_four_tokens(kind):
+def test_gpu_forward_config2_four_tokens(kind, mode):
     """Speculative verify: 4 tokens through the E = 512 layer in one call,
     i.i.d. or 4 copies of one vector + N(0, 0.1^2) noise; also equal to 4
     single-token calls."""
@@ -238,16 +249,36 @@ def test_gpu_forward_config2_four_tokens(kind):
             x = synth.hidden_states(0, 2000, 4, H0)
         else:
             x = synth.hidden_states_clustered(0, 2001, 4, H0)
-        ids, w, counts, y, dbg = _run(L, x)
+        ids, w, counts, y, dbg = _run(L, x, mode=mode)
         ref = _oracle(L, x)
         check_route(ids, w, counts, ref)
         check_forward(y, dbg, ref)
         distinct = len(set(ref["ids"].ravel().tolist()))
         assert distinct <= 32
         for t in range(4):
-            i1, w1, c1, y1, _ = _run(L, x[t:t + 1], debug=False)
+            i1, w1, c1, y1, _ = _run(L, x[t:t + 1], debug=False, mode=mode)
             assert np.array_equal(i1.cpu().numpy()[0], ids.cpu().numpy()[t])
             assert np.array_equal(u16(y1)[0], u16(y)[t])
+    finally:
+        L.close()
+
+
+def test_gpu_fused_equals_split_and_repeats():
+    """moe_decode gives the routing and output of moe_route + moe_forward, and
+    the same output again on back-to-back calls (its counters and
+    accumulators reset themselves)."""
+    L = GpuLayer(0, 5, 512, bias=True)
+    try:
+        for step in range(3):
+            x = synth.hidden_states(0, 3000 + step, 1 + step, H0)
+            a = _run(L, x, debug=False, mode="split")
+            b = _run(L, x, debug=False, mode="fused")
+            c = _run(L, x, debug=False, mode="fused")
+            for r in (b, c):
+                assert np.array_equal(a[0].cpu().numpy(), r[0].cpu().numpy())
+                assert np.array_equal(a[1].cpu().numpy(), r[1].cpu().numpy())
+                assert np.array_equal(a[2].cpu().numpy(), r[2].cpu().numpy())
+                assert np.array_equal(u16(a[3]), u16(r[3]))
     finally:
         L.close()
 

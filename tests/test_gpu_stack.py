@@ -1,0 +1,146 @@
+"""GPU parity of the layer stack (moe_stack_decode: every layer of a chained
+stack in one persistent launch).
+
+Checks: (1) the stack gives bit for bit what the same layers give one call
+at a time (moe_decode + moe_residual_rmsnorm); (2) against the float64
+oracle with teacher forcing -- each layer's routing from the GPU's own input
+x of that layer is bit-exact, and the chain's next input follows the
+oracle's residual + RMS normalisation within the layer tolerance; (3) back
+to back calls repeat (the counters and accumulators reset themselves)."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_expert_layers_b200 as moe
+import synth
+from oracle import formats as OF
+from oracle import moe as OM
+
+from moe_testlib import GpuLayer, REL_L2, to_dev_u16, u16, H0
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU collection
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+EPS = 1e-6
+
+
+def _stack_run(layers, x_bits, with_layers=True):
+    T, H = x_bits.shape
+    L = len(layers)
+    st = moe.moe_stack_create([ly.handle for ly in layers])
+    try:
+        r = to_dev_u16(x_bits)
+        x = to_dev_u16(x_bits)
+        k = layers[0].k
+        ids = torch.empty((L, T, k), dtype=torch.int32, device="cuda")
+        w = torch.empty((L, T, k), dtype=torch.float32, device="cuda")
+        xl = torch.empty((L, T, H), dtype=torch.int16, device="cuda") if with_layers else None
+        moe.moe_stack_decode(st, r, x, T, EPS, ids, w, xl)
+        torch.cuda.synchronize()
+        assert moe.moe_stack_device_error(st) == moe.MOE_OK
+        return u16(r), u16(x), ids.cpu().numpy(), w.cpu().numpy(), (u16(xl) if with_layers else None)
+    finally:
+        moe.moe_stack_destroy(st)
+
+
+def _layer_by_layer(layers, x_bits):
+    T, H = x_bits.shape
+    r = to_dev_u16(x_bits)
+    x = to_dev_u16(x_bits)
+    ids_all, w_all, x_all = [], [], []
+    for ly in layers:
+        x_all.append(u16(x))
+        ids, w, counts, y, _ = ly.decode(x, T, debug=False)
+        ids_all.append(ids.cpu().numpy())
+        w_all.append(w.cpu().numpy())
+        moe.moe_residual_rmsnorm(r, y, x, T, H, EPS)
+    torch.cuda.synchronize()
+    for ly in layers:
+        assert moe.moe_device_error(ly.handle) == moe.MOE_OK
+    return u16(r), u16(x), np.stack(ids_all), np.stack(w_all), np.stack(x_all)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_gpu_stack_equals_layer_by_layer(T):
+    """3 chained E = 512 layers (Zipf router bias): one persistent launch
+    against one moe_decode + one moe_residual_rmsnorm per layer."""
+    layers = [GpuLayer(0, 40 + l, 512, bias=True) for l in range(3)]
+    try:
+        for step in range(2):
+            x0 = synth.hidden_states(0, 4000 + 10 * T + step, T, H0)
+            a = _stack_run(layers, x0)
+            b = _layer_by_layer(layers, x0)
+            for got, ref, name in zip(a, b, ("r", "x", "ids", "w", "x_layers")):
+                assert np.array_equal(got, ref), name
+    finally:
+        for ly in layers:
+            ly.close()
+
+
+def test_gpu_stack_matches_oracle_teacher_forced():
+    """4 chained E = 32 layers, T = 2: per layer, the oracle run on the GPU's
+    own input of that layer routes identically, and the GPU's next input is
+    the oracle's residual + RMS normalisation of the oracle's y."""
+    T, L = 2, 4
+    layers = [GpuLayer(1, 60 + l, 32, bias=True) for l in range(L)]
+    try:
+        x0 = synth.hidden_states(1, 77, T, H0)
+        r_g, x_g, ids_g, w_g, xl = _stack_run(layers, x0)
+        r = x0.copy()
+        for l in range(L):
+            ref = OM.moe_layer(xl[l], layers[l].host, 32, 8, layers[l].I, 1)
+            assert np.array_equal(ids_g[l], ref["ids"]), l
+            assert np.allclose(w_g[l], ref["w"], rtol=1e-6, atol=1e-7)
+            r, x_next = OM.residual_rmsnorm(r, ref["y"], EPS)
+            got = xl[l + 1] if l + 1 < L else x_g
+            xg, xr = OF.bf16_to_f64(got), OF.bf16_to_f64(x_next)
+            rel = np.linalg.norm(xg - xr) / np.linalg.norm(xr)
+            assert rel <= REL_L2, (l, rel)
+        rg, rr = OF.bf16_to_f64(r_g), OF.bf16_to_f64(r)
+        assert np.linalg.norm(rg - rr) / np.linalg.norm(rr) <= REL_L2
+    finally:
+        for ly in layers:
+            ly.close()
+
+
+def test_gpu_stack_repeats_and_single_layer():
+    """Back-to-back calls give the same result; a one-layer stack equals
+    moe_decode followed by moe_residual_rmsnorm."""
+    layers = [GpuLayer(2, 80 + l, 32) for l in range(2)]
+    try:
+        x0 = synth.hidden_states(2, 5, 3, H0)
+        first = _stack_run(layers, x0, with_layers=False)
+        second = _stack_run(layers, x0, with_layers=False)
+        for a, b in zip(first[:4], second[:4]):
+            assert np.array_equal(a, b)
+        one = _stack_run(layers[:1], x0)
+        ref = _layer_by_layer(layers[:1], x0)
+        for got, want in zip(one, ref):
+            assert np.array_equal(got, want)
+    finally:
+        for ly in layers:
+            ly.close()
+
+
+def test_gpu_stack_argument_errors():
+    layers = [GpuLayer(3, 0, 8, 128, 64, k=2, fill="host")]
+    other = GpuLayer(3, 1, 8, 128, 128, k=2, fill="host")
+    try:
+        with pytest.raises(moe.MoEError) as ei:
+            moe.moe_stack_create([layers[0].handle, other.handle])
+        assert ei.value.code == moe.MOE_ERR_SHAPE
+        st = moe.moe_stack_create([layers[0].handle])
+        try:
+            r = to_dev_u16(np.zeros((8, 128), np.uint16))
+            x = to_dev_u16(np.zeros((8, 128), np.uint16))
+            for T in (0, 5):
+                with pytest.raises(moe.MoEError) as ei:
+                    moe.moe_stack_decode(st, r, x, T)
+                assert ei.value.code == moe.MOE_ERR_ARG
+        finally:
+            moe.moe_stack_destroy(st)
+    finally:
+        layers[0].close()
+        other.close()
