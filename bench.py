@@ -42,7 +42,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42"])
+    p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42", "prefill512"])
     p.add_argument("--layers", type=int, default=64)
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -410,10 +410,126 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------ prefill workload --
+def run_prefill(args):
+    """Chunked prefill: 512 tokens per call through an E = 512 layer with the
+    Zipf(1.1) router bias (routing + dispatch + grouped GEMMs + combine)."""
+    import torch
+    import torch.distributed as dist
+    import mxfp4_expert_layers_b200 as moe
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    moe.load()
+    hbm_peak, peak_kind = peaks()
+    T = 512
+    layers = Layers(min(args.layers, 4), bias=True, max_tokens=T)
+    L = layers.n
+    xs_host = np.stack([synth.hidden_states(0, 20000 + 7919 * rank + i, T, H) for i in range(4)])
+    xs = torch.from_numpy(xs_host.view(np.int16)).cuda()
+    ids = torch.empty((T, K_TOP), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, K_TOP), dtype=torch.float32, device="cuda")
+    counts = torch.empty((E,), dtype=torch.int32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, s):
+        moe.moe_decode(layers.handles[i % L], xs[i % xs.shape[0]], T, ids, wts, y, counts, None, s)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i, stream)
+    barrier()
+    assert all(moe.moe_device_error(h) == moe.MOE_OK for h in layers.handles)
+    touched = int((counts.cpu().numpy() > 0).sum()) + N_SHARED
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(args.steps):
+                step(args.warmup + i, cap)
+    g.replay()
+    barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    g.replay()
+    ev1.record(stream)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    # grouped GEMM kernels alone (gate/up .. down), events around them
+    for h in layers.handles:
+        moe.moe_profile_begin(h, args.steps + 2)
+    barrier()
+    for i in range(args.warmup, args.warmup + args.steps):
+        step(i, stream)
+    barrier()
+    gm_ms, gm_n = 0.0, 0
+    for h in layers.handles:
+        t_ms, n = moe.moe_profile_end(h).get("grouped_gemm", (0.0, 0))
+        gm_ms, gm_n = gm_ms + t_ms, gm_n + n
+    gemm_us = 1e3 * gm_ms / max(gm_n, 1)
+    call_us = 1e3 * ms / args.steps
+    flops = 2.0 * 3 * H * I * T * (K_TOP + N_SHARED)
+    bytes_ = touched * BYTES_PER_EXPERT + E * H * 2 + T * H * (2 + 1 + 2)
+    fp8_peak = peaks_bf16() * 2.0
+    line = {"metric": METRIC, "value": call_us / T, "unit": "us/token (512-token prefill call)", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e2m1 x e4m3 operands, f32 block sums, f64 accumulation",
+            "data": "synthetic (seeded SplitMix64 weights, Irwin-Hall normals)",
+            "config": {"workload": "chunked prefill: 512 tokens per call, E=512 top-8 + 1 shared, Zipf(1.1) bias",
+                       "layers_resident": L, "l2": "inputs larger than L2 (touched experts ~%d MB per call)" % (bytes_ // 1e6)},
+            "us_per_call": call_us, "experts_touched": touched, "flops_per_call": flops, "bytes_per_call": bytes_,
+            "roofline": {"bound": "tensor", "kernel": "gateup_kernel+down_kernel", "achieved": flops / (gemm_us * 1e6),
+                         "peak": fp8_peak, "unit": "TFLOP/s",
+                         "peak_kind": "measured bf16 cuBLAS burst x 2 (nominal fp8/bf16 ratio)",
+                         "frac": flops / (gemm_us * 1e6) / fp8_peak, "traffic": None,
+                         "hbm_gbs_of_call": bytes_ / (call_us * 1e3), "avg_launch_us": gemm_us},
+            "cpu_baseline": None, "gpu_launches": args.steps * 9, "clocks": clk,
+            "timing": "CUDA graph of K calls (route + dispatch + grouped GEMMs + combine)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    layers.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def peaks_bf16():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefill512":
+        run_prefill(args)
     else:
         run_ours(args)
 

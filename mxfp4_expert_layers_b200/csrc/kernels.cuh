@@ -81,6 +81,39 @@ bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget);
 cudaError_t launch_decode(const DecodeArgs& a, int n_ctas, cudaStream_t stream);
 int decode_static_smem();
 
+// Many-token path, T > MOE_GEMV_MAX_TOKENS (prefill.cu): dispatch and
+// grouped GEMMs over the experts that received tokens.
+struct PrefillArgs {
+  int H, I, E, k, n_shared, T;
+  const uint16_t* x;        // [T][H]
+  const int32_t* ids;       // [T][k]
+  const float* w;           // [T][k]
+  const uint8_t* w13;       // packed gate/up tiles
+  const uint8_t* w2;        // packed down tiles
+  uint16_t* y;              // [T][H]
+  // workspace (sized for max_tokens); P = T * (k + n_shared) pairs at most
+  uint8_t* xq;              // [T][H] FP8 codes (fragment order)
+  float* xs;                // [T]
+  int* counts;              // [E + S]
+  int* offsets;             // [E + S + 1]
+  int* cursor;              // [E + S]
+  int* order;               // [E + S] experts by descending count
+  int* n_active;            // [1]
+  int* n_pairs;             // [1]
+  int* queue;               // [2] work queue heads
+  int* pair_tok;            // [P]
+  float* pair_w;            // [P]
+  int* pair_ent;            // [P] position t * (k + S) + slot
+  float* h;                 // [P][I]
+  unsigned* amax;           // [P]
+  float* sh;                // [P]
+  uint8_t* qh;              // [P][I] FP8 codes (fragment order)
+  double* yacc;             // [T][H], zero between calls
+  int* err;
+  moe_debug dbg;
+};
+size_t prefill_smem_bytes(int H, int I, int which);
+
 // Optional per-kernel event timing (owned by the handle).
 struct Profiler {
   int cap = 0, n = 0;
@@ -107,6 +140,7 @@ struct PackArgs {
   uint8_t* w2_out;
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillArgs& a, int n_sms, cudaStream_t stream, Profiler* prof);
 
 // Per-row FP8 quantisation (quant.cu)
 cudaError_t launch_quantize_rows(const float* v, int rows, int cols, uint8_t* q, float* s,

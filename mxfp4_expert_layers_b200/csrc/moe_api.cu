@@ -26,6 +26,7 @@ struct moe_handle_s {
   double* yacc;        // [kMaxTokGemv][H]
   int n_sms;
   int smem_budget;     // dynamic shared memory available to the decode kernel
+  moe::PrefillArgs pf; // workspace views of the many-token path (max_tokens > 4)
   moe::Profiler prof;
   bool profiling;
 };
@@ -92,7 +93,23 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
   const size_t n_tcnt = up256(static_cast<size_t>(cfg->hidden / 16) * 4);
   const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * cfg->hidden * 8);
-  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tcnt + n_yacc;
+  // the many-token path: pairs P = max_tokens * (k + S)
+  const size_t T = static_cast<size_t>(max_tokens), H = cfg->hidden, NE = E + cfg->n_shared;
+  const size_t P = T * (cfg->top_k + cfg->n_shared);
+  const bool many = max_tokens > MOE_GEMV_MAX_TOKENS;
+  const size_t pf_sizes[] = {up256(T * H),                   // xq
+                             up256(T * 4),                   // xs
+                             up256(NE * 4), up256((NE + 1) * 4), up256(NE * 4), up256(NE * 4),  // counts offsets cursor order
+                             256,                            // n_active, n_pairs, queue
+                             up256(P * 4), up256(P * 4), up256(P * 4),   // pair_tok pair_w pair_ent
+                             up256(P * I * 4),               // h
+                             up256(P * 4), up256(P * 4),     // amax sh
+                             up256(P * I),                   // qh
+                             up256(T * H * 8)};              // yacc
+  size_t n_pf = 0;
+  if (many)
+    for (size_t v : pf_sizes) n_pf += v;
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tcnt + n_yacc + n_pf;
   int dev = 0, optin = 0;
   const int static_smem = moe::decode_static_smem();
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -122,7 +139,29 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->h = reinterpret_cast<float*>(p); p += n_h;
   h->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
   h->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
-  h->yacc = reinterpret_cast<double*>(p);
+  h->yacc = reinterpret_cast<double*>(p); p += n_yacc;
+  h->pf = moe::PrefillArgs{};
+  if (many) {
+    moe::PrefillArgs& f = h->pf;
+    size_t i = 0;
+    f.xq = p; p += pf_sizes[i++];
+    f.xs = reinterpret_cast<float*>(p); p += pf_sizes[i++];
+    f.counts = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.offsets = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.cursor = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.order = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.n_active = reinterpret_cast<int*>(p);
+    f.n_pairs = reinterpret_cast<int*>(p + 64);
+    f.queue = reinterpret_cast<int*>(p + 128); p += pf_sizes[i++];
+    f.pair_tok = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.pair_w = reinterpret_cast<float*>(p); p += pf_sizes[i++];
+    f.pair_ent = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.h = reinterpret_cast<float*>(p); p += pf_sizes[i++];
+    f.amax = reinterpret_cast<unsigned*>(p); p += pf_sizes[i++];
+    f.sh = reinterpret_cast<float*>(p); p += pf_sizes[i++];
+    f.qh = p; p += pf_sizes[i++];
+    f.yacc = reinterpret_cast<double*>(p); p += pf_sizes[i++];
+  }
   *out = h;
   return MOE_OK;
 }
@@ -174,6 +213,20 @@ int decode_call(moe_handle h, const uint16_t* x, int T, int route, int32_t* ids,
   return cuda_err(e);
 }
 
+// The many-token path: dispatch + grouped GEMMs (several launches).
+int prefill_call(moe_handle h, const uint16_t* x, int T, const int32_t* ids, const float* w, uint16_t* y,
+                 const moe_debug* dbg, cudaStream_t stream) {
+  if (!h->pf.xq) return MOE_ERR_UNSUPPORTED;  // handle created for at most MOE_GEMV_MAX_TOKENS tokens
+  const moe_config& c = h->cfg;
+  moe::PrefillArgs a = h->pf;
+  a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
+  a.x = x; a.ids = ids; a.w = w; a.w13 = h->w.w13; a.w2 = h->w.w2; a.y = y;
+  a.err = h->err;
+  if (dbg) a.dbg = *dbg;
+  h->last_path = 2;
+  return cuda_err(moe::launch_prefill(a, h->n_sms, stream, h->profiling ? &h->prof : nullptr));
+}
+
 }  // namespace
 
 int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
@@ -181,7 +234,7 @@ int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
   if (!h || !x || !topk_ids || !topk_w || !y) return MOE_ERR_ARG;
   if (T < 1 || T > h->max_tokens) return MOE_ERR_ARG;
   if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y)) return MOE_ERR_ALIGN;
-  if (T > MOE_GEMV_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+  if (T > MOE_GEMV_MAX_TOKENS) return prefill_call(h, x, T, topk_ids, topk_w, y, dbg, stream);
   return decode_call(h, x, T, 0, const_cast<int32_t*>(topk_ids), const_cast<float*>(topk_w), nullptr, y, dbg,
                      stream);
 }
@@ -193,7 +246,10 @@ int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float*
   if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y) ||
       (expert_counts && !aligned4(expert_counts)))
     return MOE_ERR_ALIGN;
-  if (T > MOE_GEMV_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+  if (T > MOE_GEMV_MAX_TOKENS) {
+    const int rc = moe_route(h, x, T, topk_ids, topk_w, expert_counts, stream);
+    return rc ? rc : prefill_call(h, x, T, topk_ids, topk_w, y, dbg, stream);
+  }
   return decode_call(h, x, T, 1, topk_ids, topk_w, expert_counts, y, dbg, stream);
 }
 
