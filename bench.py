@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42", "prefill512"])
     p.add_argument("--layers", type=int, default=64)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--prefill-kernel", default="auto", choices=["auto", "tcgen05", "exact"],
+                   help="grouped-GEMM kernels of the prefill512 workload")
     return p.parse_args()
 
 
@@ -431,6 +433,10 @@ def run_prefill(args):
     T = 512
     layers = Layers(min(args.layers, 4), bias=True, max_tokens=T)
     L = layers.n
+    kind = {"auto": moe.MOE_PREFILL_AUTO, "tcgen05": moe.MOE_PREFILL_TCGEN05,
+            "exact": moe.MOE_PREFILL_EXACT}[args.prefill_kernel]
+    for h in layers.handles:
+        moe.moe_set_prefill_kernel(h, kind)
     xs_host = np.stack([synth.hidden_states(0, 20000 + 7919 * rank + i, T, H) for i in range(4)])
     xs = torch.from_numpy(xs_host.view(np.int16)).cuda()
     ids = torch.empty((T, K_TOP), dtype=torch.int32, device="cuda")
@@ -453,6 +459,7 @@ def run_prefill(args):
     barrier()
     assert all(moe.moe_device_error(h) == moe.MOE_OK for h in layers.handles)
     touched = int((counts.cpu().numpy() > 0).sum()) + N_SHARED
+    tc = moe.moe_last_path(layers.handles[0]) == 3
     g = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
@@ -496,12 +503,16 @@ def run_prefill(args):
     line = {"metric": METRIC, "value": call_us / T, "unit": "us/token (512-token prefill call)", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "e2m1 x e4m3 operands, f32 block sums, f64 accumulation",
+            "dtype": ("e2m1 x e4m3 operands (tcgen05 block-scaled MMA), f32 accumulation" if tc else
+                      "e2m1 x e4m3 operands, f32 block sums, f64 accumulation"),
             "data": "synthetic (seeded SplitMix64 weights, Irwin-Hall normals)",
             "config": {"workload": "chunked prefill: 512 tokens per call, E=512 top-8 + 1 shared, Zipf(1.1) bias",
                        "layers_resident": L, "l2": "inputs larger than L2 (touched experts ~%d MB per call)" % (bytes_ // 1e6)},
             "us_per_call": call_us, "experts_touched": touched, "flops_per_call": flops, "bytes_per_call": bytes_,
-            "roofline": {"bound": "tensor", "kernel": "gateup_kernel+down_kernel", "achieved": flops / (gemm_us * 1e6),
+            "roofline": {"bound": "tensor",
+                         "kernel": ("tc_gemm_kernel<0>+requant_kernel+tc_gemm_kernel<1>" if tc else
+                                    "gateup_kernel+requant_kernel+down_kernel"),
+                         "achieved": flops / (gemm_us * 1e6),
                          "peak": fp8_peak, "unit": "TFLOP/s",
                          "peak_kind": "measured bf16 cuBLAS burst x 2 (nominal fp8/bf16 ratio)",
                          "frac": flops / (gemm_us * 1e6) / fp8_peak, "traffic": None,

@@ -232,8 +232,28 @@ int moe_stack_destroy(moe_stack s);
 int moe_device_error(moe_handle h, cudaStream_t stream);
 
 /* Which kernel path the last moe_forward on this handle launched:
- * 1 = GEMV (T <= MOE_GEMV_MAX_TOKENS), 2 = grouped GEMM, 0 = none yet. */
+ * 1 = fused decode kernel (T <= MOE_GEMV_MAX_TOKENS), 2 = grouped GEMM on
+ * mma.sync with exact block sums, 3 = grouped GEMM on tcgen05 (block-scaled
+ * MMA, float32 accumulation in tensor memory), 0 = none yet. */
 int moe_last_path(moe_handle h);
+
+/* Kernels of the many-token path (T > MOE_GEMV_MAX_TOKENS).
+ *   MOE_PREFILL_AUTO    tcgen05 grouped GEMMs when the shape allows them
+ *                       (hidden a multiple of 128),
+ *                       else the mma.sync kernels (the default);
+ *   MOE_PREFILL_TCGEN05 always the tcgen05 kernels (MOE_ERR_UNSUPPORTED if
+ *                       the shape does not allow them);
+ *   MOE_PREFILL_EXACT   the mma.sync kernels, whose 32-element block sums are
+ *                       exact and scaled and summed in float64 like the decode
+ *                       kernel's (h then matches the float64 definition up to
+ *                       its final rounding to float32).
+ * The tcgen05 kernels sum the scaled block products in float32 inside the
+ * tensor cores, so h carries float32 rounding of the K-long sum.
+ * Errors: MOE_ERR_ARG (bad handle or kind), MOE_ERR_UNSUPPORTED. */
+#define MOE_PREFILL_AUTO 0
+#define MOE_PREFILL_TCGEN05 1
+#define MOE_PREFILL_EXACT 2
+int moe_set_prefill_kernel(moe_handle h, int kind);
 
 /* Per-kernel timing.  moe_profile_begin(h, n) makes the following calls on
  * this handle record a CUDA event pair around each kernel they launch (up to

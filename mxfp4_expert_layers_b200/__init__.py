@@ -24,8 +24,12 @@ MOE_ERR_TIMEOUT = -5
 MOE_ERR_UNSUPPORTED = -6
 MOE_ERR_DEVICE = -7
 MOE_GEMV_MAX_TOKENS = 4
+MOE_PREFILL_AUTO = 0
+MOE_PREFILL_TCGEN05 = 1
+MOE_PREFILL_EXACT = 2
 
 EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
+           "moe_set_prefill_kernel",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
            "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static",
            "moe_decode", "moe_stack_create", "moe_stack_decode", "moe_stack_device_error",
@@ -86,6 +90,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_decode.argtypes = [p, p, i, p, p, p, p, ctypes.POINTER(moe_debug), p]
     L.moe_device_error.argtypes = [p, p]
     L.moe_last_path.argtypes = [p]
+    L.moe_set_prefill_kernel.argtypes = [p, i]
     L.moe_destroy.argtypes = [p]
     L.moe_stack_create.argtypes = [p, i, p]
     L.moe_stack_decode.argtypes = [p, p, p, i, ctypes.c_float, p, p, p, p]
@@ -204,6 +209,11 @@ def moe_device_error(handle: int, stream=None) -> int:
 
 def moe_last_path(handle: int) -> int:
     return load().moe_last_path(handle)
+
+
+def moe_set_prefill_kernel(handle: int, kind: int) -> None:
+    """Kernels of the many-token path: MOE_PREFILL_AUTO, _TCGEN05 or _EXACT."""
+    _check(load().moe_set_prefill_kernel(handle, kind), "moe_set_prefill_kernel")
 
 
 def moe_destroy(handle: int) -> None:

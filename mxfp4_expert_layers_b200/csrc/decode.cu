@@ -192,8 +192,14 @@ __device__ __forceinline__ void build_distinct(const int32_t* ids, const float* 
 
 // A bounded wait gave up: say where (the error word reports it to the host).
 __device__ __noinline__ void note_timeout(int line, int layer, int entry) {
+#ifdef MOE_TRACE
   printf("decode_kernel: bounded wait gave up (source line %d, CTA %d, layer %d, entry %d)\n", line, blockIdx.x,
          layer, entry);
+#else
+  (void)line;
+  (void)layer;
+  (void)entry;
+#endif
 }
 
 // CTA owning down slab q: the largest c with floor(c * S / G) <= q.
@@ -536,20 +542,23 @@ decode_kernel(DecodeArgs a) {
       for (int j = npre + warp; j < min(ng, NG); j += kWarps) issue_gu(a, sm, lw, dist.expert, j, gu_base + j);
       for (int i = warp; i < min(nq, ND); i += kWarps) issue_dn(a, sm, lw, dist.expert, nd, q0 + i, dn_base + i);
     }
-    // pair table of the down step (off the critical path)
-    if (warp == kWarps - 1 && lane == 0) {
-      int np = 0;
-      for (int u = 0; u < nd; ++u)
-        for (int t = 0; t < kMaxTokGemv; ++t) {
-          const bool use = t < T && (dist.mask[u] >> t & 1);
-          pair_of[u][t] = use ? np : -1;
-          if (use) {
-            pair_d[np] = u;
-            pair_t[np] = t;
-            ++np;
-          }
+    // pair table of the down step (off the critical path): the (expert,
+    // token) pairs in order, numbered by a ballot prefix count
+    if (warp == kWarps - 1) {
+      int base_p = 0;
+      for (int i0 = 0; i0 < kMaxDistinct * kMaxTokGemv; i0 += 32) {
+        const int i = i0 + lane, u = i / kMaxTokGemv, t = i % kMaxTokGemv;
+        const bool use = u < nd && t < T && (dist.mask[u] >> t & 1);
+        const unsigned m = __ballot_sync(0xffffffffu, use);
+        const int pi = base_p + __popc(m & ((1u << lane) - 1u));
+        if (u < kMaxDistinct) pair_of[u][t] = use ? pi : -1;
+        if (use) {
+          pair_d[pi] = u;
+          pair_t[pi] = t;
         }
-      s_npairs = np;
+        base_p += __popc(m);
+      }
+      if (lane == 0) s_npairs = base_p;
     }
     MOE_TRACE_POINT(3, 6);
 
@@ -677,32 +686,37 @@ decode_kernel(DecodeArgs a) {
         const int u = i / kMaxTokGemv, tt = i % kMaxTokGemv;
         if (pair_of[u][tt] < 0) coef[u][tt] = 0.0;
       }
-      // h of every pair -> registers (4 floats per load, up to 8 in flight)
+      // h of every pair -> registers (4 floats per load, 4 loads in flight),
+      // then FP8 codes in the fragment order (each group of 8 elements holds
+      // its even elements, then its odd ones)
       const int per = I / 4;
       const int total4 = np * per;
-      for (int b4 = 0; b4 < total4; b4 += 8 * kThreads) {
-        float4 v[8];
+      __syncthreads();  // scales visible
+      for (int b4 = 0; b4 < total4; b4 += 4 * kThreads) {
+        float4 v[4];
+        int pr[4];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < 4; ++r) {
           const int idx = b4 + tid + r * kThreads;
-          if (idx < total4) {
-            const int p = idx / per, j4 = idx % per;
+          pr[r] = idx < total4 ? idx / per : -1;
+          if (pr[r] >= 0)
             v[r] = __ldcg(reinterpret_cast<const float4*>(
-                              a.h + (static_cast<size_t>(pair_d[p]) * kMaxTokGemv + pair_t[p]) * I) + j4);
-          }
+                              a.h + (static_cast<size_t>(pair_d[pr[r]]) * kMaxTokGemv + pair_t[pr[r]]) * I) +
+                          (idx - pr[r] * per));
         }
-        __syncthreads();  // scales visible
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int idx = b4 + tid + r * kThreads;
-          if (idx < total4) {
-            const int p = idx / per, j = 4 * (idx % per);
-            const float shv = shs[pair_d[p]][pair_t[p]];
-            const float hv[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-            uint8_t* row = qh + static_cast<size_t>(p) * I + (j & ~31);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) row[perm_pos((j & 31) + q)] = f32_to_e4m3(__fdiv_rn(hv[q], shv));
-          }
+        for (int r = 0; r < 4; ++r) {
+          if (pr[r] < 0) continue;
+          const int j = 4 * (b4 + tid + r * kThreads - pr[r] * per);
+          const float shv = shs[pair_d[pr[r]]][pair_t[pr[r]]];
+          const uint32_t c0 = f32_to_e4m3(__fdiv_rn(v[r].x, shv)), c1 = f32_to_e4m3(__fdiv_rn(v[r].y, shv));
+          const uint32_t c2 = f32_to_e4m3(__fdiv_rn(v[r].z, shv)), c3 = f32_to_e4m3(__fdiv_rn(v[r].w, shv));
+          // elements j..j+3 (j % 4 == 0): the two even ones go to bytes
+          // o, o+1 of the group's even half, the two odd ones to the odd half
+          uint8_t* grp = qh + static_cast<size_t>(pr[r]) * I + (j & ~7);
+          const int o = (j & 4) >> 1;
+          *reinterpret_cast<uint16_t*>(grp + o) = static_cast<uint16_t>(c0 | c2 << 8);
+          *reinterpret_cast<uint16_t*>(grp + 4 + o) = static_cast<uint16_t>(c1 | c3 << 8);
         }
       }
       __syncthreads();

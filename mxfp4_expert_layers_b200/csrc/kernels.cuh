@@ -30,6 +30,9 @@ struct RouteArgs {
   const uint8_t* w13;   // packed
   const uint8_t* w2;    // packed
 };
+// T > kRouteGemmMinTokens: logits GEMM on the FP64 tensor-core path + a
+// top-k kernel; otherwise one fused launch (programmatic dependent launch).
+constexpr int kRouteGemmMinTokens = 32;
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 int route_tiles(int T);
 
@@ -91,28 +94,53 @@ struct PrefillArgs {
   const uint8_t* w13;       // packed gate/up tiles
   const uint8_t* w2;        // packed down tiles
   uint16_t* y;              // [T][H]
+  int tc;                   // 1: tcgen05 grouped GEMMs, 0: mma.sync with exact block sums
   // workspace (sized for max_tokens); P = T * (k + n_shared) pairs at most
   uint8_t* xq;              // [T][H] FP8 codes (fragment order)
   float* xs;                // [T]
   int* counts;              // [E + S]
-  int* offsets;             // [E + S + 1]
+  int* offsets;             // [E + S + 1] first pair of each expert
+  int* roff;                // [E + S + 1] first operand-panel row of each expert (counts rounded up to 8)
   int* cursor;              // [E + S]
-  int* order;               // [E + S] experts by descending count
+  int* order;               // [E + S] experts with tokens, in index order
   int* n_active;            // [1]
   int* n_pairs;             // [1]
   int* queue;               // [2] work queue heads
+  int* item_base;           // [2][kItemBaseStride] tensor-core work items before each expert rank
   int* pair_tok;            // [P]
   float* pair_w;            // [P]
   int* pair_ent;            // [P] position t * (k + S) + slot
+  int* pair_row;            // [P] operand-panel row of each pair
+  int* ent_row;             // [T * (k + S)] operand-panel row of each (token, slot), -1 if none
   float* h;                 // [P][I]
-  unsigned* amax;           // [P]
   float* sh;                // [P]
-  uint8_t* qh;              // [P][I] FP8 codes (fragment order)
-  double* yacc;             // [T][H], zero between calls
+  uint8_t* qh;              // [P][I] FP8 codes (fragment order), mma.sync kernels
+  // Operand panels of the tcgen05 kernels: FP8 codes of x (K = H) and of h
+  // (K = I) per panel row, laid out as the MMA reads them (panel_off).
+  uint8_t* xg;
+  uint8_t* qg;
+  int rcap;                 // panel rows (multiple of 8)
+  double* yacc;             // [T][H] float64 accumulator of the mma.sync kernels, zero between calls
+  float* yacc32;            // [T][H] float32 accumulator of the tcgen05 kernels (same memory), zero between calls
   int* err;
   moe_debug dbg;
 };
+
+// Byte offset of code k (fragment order) of panel row R: K is cut into
+// chunks of 256 codes; a chunk holds the rows in bands of 8, each band 16
+// pieces of 8 rows x 16 codes (the no-swizzle K-major layout of tcgen05
+// operands, 2048 bytes per band).
+__host__ __device__ inline size_t panel_off(int R, int k, int rcap) {
+  return static_cast<size_t>(k >> 8) * (static_cast<size_t>(rcap >> 3) * 2048) +
+         static_cast<size_t>(R >> 3) * 2048 + static_cast<size_t>(((k & 255) >> 4) * 128 + (R & 7) * 16 + (k & 15));
+}
 size_t prefill_smem_bytes(int H, int I, int which);
+constexpr int kItemBaseStride = MOE_MAX_EXPERTS + MOE_MAX_SHARED + 1;
+// Grouped GEMMs on tcgen05 (prefill_tc.cu): shapes they take, shared memory,
+// launch of projection `which` (0 gate/up + SwiGLU, 1 down + combine).
+bool prefill_tc_supported(int H, int I);
+size_t prefill_tc_smem_bytes();
+cudaError_t launch_prefill_tc(const PrefillArgs& a, int n_sms, cudaStream_t stream, int which);
 
 // Optional per-kernel event timing (owned by the handle).
 struct Profiler {
@@ -140,6 +168,8 @@ struct PackArgs {
   uint8_t* w2_out;
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t stream);
+// a.tc selects the grouped GEMMs on tcgen05 (needs prefill_tc_supported);
+// otherwise the mma.sync kernels with the decode path's exact block sums.
 cudaError_t launch_prefill(const PrefillArgs& a, int n_sms, cudaStream_t stream, Profiler* prof);
 
 // Per-row FP8 quantisation (quant.cu)

@@ -12,6 +12,7 @@ struct moe_handle_s {
   moe_weights w;
   int max_tokens;
   int last_path;
+  int prefill_kernel;  // MOE_PREFILL_*
   void* ws;
   size_t ws_bytes;
   // workspace views
@@ -97,15 +98,23 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const size_t T = static_cast<size_t>(max_tokens), H = cfg->hidden, NE = E + cfg->n_shared;
   const size_t P = T * (cfg->top_k + cfg->n_shared);
   const bool many = max_tokens > MOE_GEMV_MAX_TOKENS;
+  // operand panels of the tcgen05 kernels: rows = pairs with every expert's
+  // count rounded up to 8; K cut into chunks of 256 codes, 2048 bytes per band
+  const size_t rcap = (P + 7) / 8 * 8 + 8 * NE;
+  const size_t xg_bytes = (H + 255) / 256 * (rcap / 8) * 2048, qg_bytes = (I + 255) / 256 * (rcap / 8) * 2048;
   const size_t pf_sizes[] = {up256(T * H),                   // xq
                              up256(T * 4),                   // xs
-                             up256(NE * 4), up256((NE + 1) * 4), up256(NE * 4), up256(NE * 4),  // counts offsets cursor order
+                             up256(NE * 4), up256((NE + 1) * 4), up256((NE + 1) * 4),  // counts offsets roff
+                             up256(NE * 4), up256(NE * 4),   // cursor order
                              256,                            // n_active, n_pairs, queue
-                             up256(P * 4), up256(P * 4), up256(P * 4),   // pair_tok pair_w pair_ent
+                             up256(P * 4), up256(P * 4), up256(P * 4), up256(P * 4),  // pair_tok pair_w pair_ent pair_row
+                             up256(P * 4),                   // ent_row
                              up256(P * I * 4),               // h
-                             up256(P * 4), up256(P * 4),     // amax sh
+                             up256(P * 4),                   // sh
                              up256(P * I),                   // qh
-                             up256(T * H * 8)};              // yacc
+                             up256(T * H * 8),               // yacc (float64; float32 view for tcgen05)
+                             up256(2 * moe::kItemBaseStride * 4),  // item_base
+                             up256(xg_bytes), up256(qg_bytes)};    // xg qg
   size_t n_pf = 0;
   if (many)
     for (size_t v : pf_sizes) n_pf += v;
@@ -148,6 +157,7 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     f.xs = reinterpret_cast<float*>(p); p += pf_sizes[i++];
     f.counts = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.offsets = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.roff = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.cursor = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.order = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.n_active = reinterpret_cast<int*>(p);
@@ -156,11 +166,17 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     f.pair_tok = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.pair_w = reinterpret_cast<float*>(p); p += pf_sizes[i++];
     f.pair_ent = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.pair_row = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.ent_row = reinterpret_cast<int*>(p); p += pf_sizes[i++];
     f.h = reinterpret_cast<float*>(p); p += pf_sizes[i++];
-    f.amax = reinterpret_cast<unsigned*>(p); p += pf_sizes[i++];
     f.sh = reinterpret_cast<float*>(p); p += pf_sizes[i++];
     f.qh = p; p += pf_sizes[i++];
-    f.yacc = reinterpret_cast<double*>(p); p += pf_sizes[i++];
+    f.yacc = reinterpret_cast<double*>(p);
+    f.yacc32 = reinterpret_cast<float*>(p); p += pf_sizes[i++];
+    f.item_base = reinterpret_cast<int*>(p); p += pf_sizes[i++];
+    f.xg = p; p += pf_sizes[i++];
+    f.qg = p; p += pf_sizes[i++];
+    f.rcap = static_cast<int>(rcap);
   }
   *out = h;
   return MOE_OK;
@@ -223,7 +239,10 @@ int prefill_call(moe_handle h, const uint16_t* x, int T, const int32_t* ids, con
   a.x = x; a.ids = ids; a.w = w; a.w13 = h->w.w13; a.w2 = h->w.w2; a.y = y;
   a.err = h->err;
   if (dbg) a.dbg = *dbg;
-  h->last_path = 2;
+  const bool tc = h->prefill_kernel != MOE_PREFILL_EXACT && moe::prefill_tc_supported(c.hidden, c.inter);
+  if (h->prefill_kernel == MOE_PREFILL_TCGEN05 && !tc) return MOE_ERR_UNSUPPORTED;
+  a.tc = tc ? 1 : 0;
+  h->last_path = tc ? 3 : 2;
   return cuda_err(moe::launch_prefill(a, h->n_sms, stream, h->profiling ? &h->prof : nullptr));
 }
 
@@ -274,6 +293,14 @@ int moe_device_error(moe_handle h, cudaStream_t stream) {
 }
 
 int moe_last_path(moe_handle h) { return h ? h->last_path : 0; }
+
+int moe_set_prefill_kernel(moe_handle h, int kind) {
+  if (!h || kind < MOE_PREFILL_AUTO || kind > MOE_PREFILL_EXACT) return MOE_ERR_ARG;
+  if (kind == MOE_PREFILL_TCGEN05 && !moe::prefill_tc_supported(h->cfg.hidden, h->cfg.inter))
+    return MOE_ERR_UNSUPPORTED;
+  h->prefill_kernel = kind;
+  return MOE_OK;
+}
 
 static void free_profiler(moe::Profiler& p) {
   for (int i = 0; i < 2 * p.cap; ++i) cudaEventDestroy(p.ev[i]);

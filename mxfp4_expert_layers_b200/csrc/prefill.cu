@@ -9,23 +9,30 @@
 // many tokens per call touch many experts -- here most of the 512.
 //
 // Kernels, in stream order:
-//  1. quantise x: FP8 E4M3 codes per token with amax/448 (fragment order).
-//  2. dispatch: counts per expert, offsets (exclusive scan), the experts in
-//     descending count order, and the pair lists (token, routing weight) of
-//     every expert; the shared experts take every token with weight 1.
-//  3. gate/up: work item = (expert, tile of 8 gate + 8 up rows), taken from a
-//     queue in descending token count; the tile is copied once into shared
-//     memory (bulk copy, the next item's tile in flight meanwhile) and used
-//     for all of the expert's tokens, 8 tokens per mma.sync m16n8k32 e4m3.
-//     Block sums are exact in float32; scaled by 2^(E-127+6) and summed in
-//     float64 (the same arithmetic as the decode path), then SwiGLU in
-//     float64 -> h (float32) per pair and the pair's amax.
-//  4. requantise h: FP8 codes per pair with amax/448.
-//  5. down: work item = (expert, tile of 16 output rows), 8 pairs per MMA;
-//     each pair's 16 outputs times w * s_h are added to a float64
-//     accumulator of the token (atomic adds; the order of the ~9 additions per
-//     output is free, which moves the float64 sum by at most a few units in
-//     its last place).
+//  1. dispatch: counts per expert; one CTA scans them into the pair offsets
+//     of every expert, its first operand-panel row (counts rounded up to 8),
+//     the experts with tokens (index order) and the first work item of each;
+//     then the pair lists (token, routing weight, panel row) of every expert.
+//     The shared experts take every token with weight 1.
+//  2. quantise x: FP8 E4M3 codes per token with amax/448 (fragment order);
+//     for the tcgen05 kernels also copied into the operand-panel row of each
+//     of the token's pairs.
+//  3. gate/up + SwiGLU -> h (float32) per pair, on one of two kernel sets:
+//     - tcgen05 (prefill_tc.cu): work item = (expert, 64 features, up to 128
+//       of its tokens), block-scaled MMA with float32 accumulation in tensor
+//       memory;
+//     - mma.sync: work item = (expert, tile of 8 gate + 8 up rows), taken
+//       from a queue; the tile is copied once into shared memory (bulk copy,
+//       the next item's tile in flight meanwhile) and used for all of the
+//       expert's tokens, 8 tokens per mma.sync m16n8k32 e4m3.  Block sums
+//       are exact in float32; scaled by 2^(E-127+6) and summed in float64
+//       (the decode path's arithmetic), then SwiGLU in float64.
+//  4. requantise h: per pair amax, s_h = amax/448 and FP8 codes (panel rows
+//     for tcgen05, plain rows for mma.sync).
+//  5. down + combine: each pair's outputs times w * s_h are added to an
+//     accumulator of its token (atomic adds; tcgen05: float32, 4 outputs per
+//     add; mma.sync: float64, tile of 16 output rows, 8 pairs per MMA).  The
+//     order of the ~9 additions per output is free.
 //  6. finalize: y = bf16(accumulator), accumulator cleared.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -71,6 +78,12 @@ __global__ void __launch_bounds__(kQThreads) quant_x_kernel(PrefillArgs a) {
   }
   __syncthreads();
   const float s = s_s;
+  // panel rows of the token's pairs (tcgen05 kernels)
+  const int ns = a.k + a.n_shared;
+  int rows[MOE_MAX_TOPK + MOE_MAX_SHARED];
+#pragma unroll
+  for (int sl = 0; sl < MOE_MAX_TOPK + MOE_MAX_SHARED; ++sl)
+    rows[sl] = a.tc && sl < ns ? __ldg(a.ent_row + static_cast<size_t>(t) * ns + sl) : -1;
   for (int u = tid; u < H / 8; u += kQThreads) {
     const uint4 v = __ldg(xr + u);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -80,8 +93,14 @@ __global__ void __launch_bounds__(kQThreads) quant_x_kernel(PrefillArgs a) {
       const float xv = __uint_as_float(jj & 1 ? (wv[jj >> 1] & 0xFFFF0000u) : (wv[jj >> 1] << 16));
       q[jj] = f32_to_e4m3(__fdiv_rn(xv, s));
     }
-    reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(t) * H)[u] =
+    const uint2 codes =
         make_uint2(q[0] | q[2] << 8 | q[4] << 16 | q[6] << 24, q[1] | q[3] << 8 | q[5] << 16 | q[7] << 24);
+    reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(t) * H)[u] = codes;
+    if (a.tc) {
+#pragma unroll
+      for (int sl = 0; sl < MOE_MAX_TOPK + MOE_MAX_SHARED; ++sl)
+        if (rows[sl] >= 0) *reinterpret_cast<uint2*>(a.xg + panel_off(rows[sl], 8 * u, a.rcap)) = codes;
+    }
     if (a.dbg.xq)
       reinterpret_cast<uint2*>(a.dbg.xq + static_cast<size_t>(t) * H)[u] =
           make_uint2(q[0] | q[1] << 8 | q[2] << 16 | q[3] << 24, q[4] | q[5] << 8 | q[6] << 16 | q[7] << 24);
@@ -99,39 +118,71 @@ __global__ void count_kernel(PrefillArgs a) {
   }
 }
 
-// One CTA: offsets, the order of the experts by descending count (ties: lower
-// index), the number with tokens, the fill cursors, and the two work queues.
+// Block-wide exclusive prefix sums of N values per thread (blockDim.x a
+// multiple of 32, at most 1024); tot receives the totals.
+template <int N>
+__device__ void block_exclusive_scan(int (&v)[N], int (&tot)[N]) {
+  __shared__ int ws[N][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int inc[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    inc[i] = v[i];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc[i], o);
+      if (lane >= o) inc[i] += y;
+    }
+    if (lane == 31) ws[i][warp] = inc[i];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      int x = lane < nw ? ws[i][lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      ws[i][lane] = x;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    v[i] = (warp > 0 ? ws[i][warp - 1] : 0) + inc[i] - v[i];
+    tot[i] = ws[i][nw - 1];
+  }
+  __syncthreads();
+}
+
+// One CTA, thread e = expert e: pair offsets and fill cursors, panel-row
+// offsets (counts rounded up to 8), the experts with tokens in index order,
+// the first work item of each (tcgen05 kernels: 64-feature gate/up tiles and
+// 128-row down tiles, times 128-token column tiles), and the work queues.
 __global__ void __launch_bounds__(1024) scan_kernel(PrefillArgs a) {
-  __shared__ int cnt[MOE_MAX_EXPERTS + MOE_MAX_SHARED];
-  __shared__ int off[MOE_MAX_EXPERTS + MOE_MAX_SHARED + 1];
-  const int NE = a.E + a.n_shared, tid = threadIdx.x;
-  for (int e = tid; e < NE; e += blockDim.x) cnt[e] = e < a.E ? a.counts[e] : a.T;
-  __syncthreads();
-  if (tid == 0) {
-    int s = 0;
-    for (int e = 0; e < NE; ++e) {
-      off[e] = s;
-      s += cnt[e];
-    }
-    off[NE] = s;
-    a.n_pairs[0] = s;
-  }
-  __syncthreads();
-  int active = 0;
-  for (int e = tid; e < NE; e += blockDim.x) {
-    a.offsets[e] = off[e];
-    a.cursor[e] = off[e];
-    if (cnt[e] > 0) {
-      int rank = 0;
-      for (int f = 0; f < NE; ++f) rank += cnt[f] > cnt[e] || (cnt[f] == cnt[e] && f < e);
-      a.order[rank] = e;
-      ++active;
+  const int NE = a.E + a.n_shared, e = threadIdx.x;
+  const int c = e < NE ? (e < a.E ? a.counts[e] : a.T) : 0;
+  const int nt = (c + 127) / 128;
+  int v[5] = {c, (c + 7) & ~7, c > 0 ? 1 : 0, nt * (a.I / 64), nt * (a.H / 128)};
+  int tot[5];
+  block_exclusive_scan<5>(v, tot);
+  if (e < NE) {
+    a.offsets[e] = v[0];
+    a.cursor[e] = v[0];
+    a.roff[e] = v[1];
+    if (c > 0) {
+      a.order[v[2]] = e;
+      a.item_base[v[2]] = v[3];
+      a.item_base[kItemBaseStride + v[2]] = v[4];
     }
   }
-  if (tid == 0) a.offsets[NE] = off[NE];
-  active = __syncthreads_count(active);
-  if (tid == 0) {
-    a.n_active[0] = active;
+  if (e == 0) {
+    a.offsets[NE] = tot[0];
+    a.roff[NE] = tot[1];
+    a.n_pairs[0] = tot[0];
+    a.n_active[0] = tot[2];
+    a.item_base[tot[2]] = tot[3];
+    a.item_base[kItemBaseStride + tot[2]] = tot[4];
     a.queue[0] = 0;  // gate/up work queue
     a.queue[1] = 0;  // down work queue
   }
@@ -144,9 +195,12 @@ __global__ void fill_kernel(PrefillArgs a) {
     float w;
     if (i < nr) {
       e = __ldg(a.ids + i);
-      if (e < 0 || e >= a.E) continue;
       t = i / a.k;
       slot = i % a.k;
+      if (e < 0 || e >= a.E) {
+        a.ent_row[t * (a.k + a.n_shared) + slot] = -1;
+        continue;
+      }
       w = __ldg(a.w + i);
     } else {
       e = a.E + (i - nr) / a.T;
@@ -158,6 +212,9 @@ __global__ void fill_kernel(PrefillArgs a) {
     a.pair_tok[p] = t;
     a.pair_w[p] = w;
     a.pair_ent[p] = t * (a.k + a.n_shared) + slot;
+    const int row = a.roff[e] + (p - a.offsets[e]);
+    a.pair_row[p] = row;
+    a.ent_row[t * (a.k + a.n_shared) + slot] = row;
   }
 }
 
@@ -252,8 +309,6 @@ __global__ void __launch_bounds__(kG1Threads, 1) gateup_kernel(PrefillArgs a) {
           const double gv = s * gs, uv = s * us;
           const float hv = static_cast<float>(gv / (1.0 + exp(-gv)) * uv);
           a.h[static_cast<size_t>(p) * I + f0 + f] = hv;
-          const float m = fabsf(hv);
-          if (m > 0.f) atomicMax(a.amax + p, __float_as_uint(m));
         }
       }
       __syncthreads();
@@ -267,21 +322,34 @@ __global__ void __launch_bounds__(kG1Threads, 1) gateup_kernel(PrefillArgs a) {
 }
 
 // --------------------------------------------------- 4. requantise h ---
+// One warp per pair: amax of its h row, s_h = amax/448, FP8 codes in the
+// fragment order (each group of 8: even elements, then odd ones), written to
+// the pair's panel row (tcgen05) or plain row (mma.sync).
 __global__ void requant_kernel(PrefillArgs a) {
-  const int P = a.n_pairs[0], I = a.I;
-  for (int p = blockIdx.x; p < P; p += gridDim.x) {
-    const float amax = __uint_as_float(a.amax[p]);
-    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-    if (threadIdx.x == 0) a.sh[p] = s;
-    for (int u = threadIdx.x; u < I / 8; u += blockDim.x) {
-      const float4 v0 = *reinterpret_cast<const float4*>(a.h + static_cast<size_t>(p) * I + 8 * u);
-      const float4 v1 = *reinterpret_cast<const float4*>(a.h + static_cast<size_t>(p) * I + 8 * u + 4);
+  const int P = a.n_pairs[0], I = a.I, lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int p = blockIdx.x * wpb + (threadIdx.x >> 5); p < P; p += gridDim.x * wpb) {
+    const float* hr = a.h + static_cast<size_t>(p) * I;
+    float m = 0.f;
+    for (int u = lane; u < I / 4; u += 32) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(hr) + u);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    m = warp_max_f32(m);
+    const float s = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+    if (lane == 0) a.sh[p] = s;
+    const int row = a.tc ? a.pair_row[p] : 0;
+    for (int u = lane; u < I / 8; u += 32) {
+      const float4 v0 = __ldcg(reinterpret_cast<const float4*>(hr + 8 * u));
+      const float4 v1 = __ldcg(reinterpret_cast<const float4*>(hr + 8 * u + 4));
       const float hv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
       uint32_t q[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) q[j] = f32_to_e4m3(__fdiv_rn(hv[j], s));
-      reinterpret_cast<uint2*>(a.qh + static_cast<size_t>(p) * I)[u] =
+      const uint2 codes =
           make_uint2(q[0] | q[2] << 8 | q[4] << 16 | q[6] << 24, q[1] | q[3] << 8 | q[5] << 16 | q[7] << 24);
+      if (a.tc) *reinterpret_cast<uint2*>(a.qg + panel_off(row, 8 * u, a.rcap)) = codes;
+      else reinterpret_cast<uint2*>(a.qh + static_cast<size_t>(p) * I)[u] = codes;
     }
   }
 }
@@ -388,7 +456,10 @@ __global__ void debug_kernel(PrefillArgs a) {
     if (threadIdx.x == 0 && a.dbg.sh) a.dbg.sh[ent] = a.sh[p];
     for (int j = threadIdx.x; j < I; j += blockDim.x) {
       if (a.dbg.h) a.dbg.h[ent * I + j] = a.h[static_cast<size_t>(p) * I + j];
-      if (a.dbg.qh) a.dbg.qh[ent * I + j] = a.qh[static_cast<size_t>(p) * I + (j & ~31) + perm_pos(j & 31)];
+      if (a.dbg.qh) {
+        const int jf = (j & ~31) + perm_pos(j & 31);
+        a.dbg.qh[ent * I + j] = a.tc ? a.qg[panel_off(a.pair_row[p], jf, a.rcap)] : a.qh[static_cast<size_t>(p) * I + jf];
+      }
     }
   }
 }
@@ -398,8 +469,13 @@ __global__ void finalize_kernel(PrefillArgs a) {
   const size_t n = static_cast<size_t>(a.T) * a.H;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    a.y[i] = f64_to_bf16_rne(a.yacc[i]);
-    a.yacc[i] = 0.0;
+    if (a.tc) {
+      a.y[i] = f64_to_bf16_rne(static_cast<double>(a.yacc32[i]));
+      a.yacc32[i] = 0.f;
+    } else {
+      a.y[i] = f64_to_bf16_rne(a.yacc[i]);
+      a.yacc[i] = 0.0;
+    }
   }
 }
 
@@ -410,28 +486,34 @@ size_t prefill_smem_bytes(int H, int I, int which) {
                     : 2 * static_cast<size_t>(dn_tile_bytes(I)) + kG2Warps * 16 * kCols * sizeof(double);
 }
 
-cudaError_t launch_prefill(const PrefillArgs& a_in, int n_sms, cudaStream_t stream, Profiler* prof) {
-  PrefillArgs a = a_in;
+cudaError_t launch_prefill(const PrefillArgs& a, int n_sms, cudaStream_t stream, Profiler* prof) {
   const size_t s1 = prefill_smem_bytes(a.H, a.I, 0), s2 = prefill_smem_bytes(a.H, a.I, 1);
-  cudaError_t err = cudaFuncSetAttribute(gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(s1));
-  if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (!a.tc) {
+    err = cudaFuncSetAttribute(gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
+    if (err != cudaSuccess) return err;
+  }
   const int NE = a.E + a.n_shared;
   if ((err = cudaMemsetAsync(a.counts, 0, static_cast<size_t>(NE) * sizeof(int), stream)) != cudaSuccess) return err;
-  if ((err = cudaMemsetAsync(a.amax, 0, static_cast<size_t>(a.T) * (a.k + a.n_shared) * sizeof(unsigned),
-                             stream)) != cudaSuccess)
-    return err;
   const int nfill = a.T * (a.k + a.n_shared);
-  quant_x_kernel<<<a.T, kQThreads, 0, stream>>>(a);
   count_kernel<<<(a.T * a.k + 255) / 256, 256, 0, stream>>>(a);
   scan_kernel<<<1, 1024, 0, stream>>>(a);
   fill_kernel<<<(nfill + 255) / 256, 256, 0, stream>>>(a);
+  quant_x_kernel<<<a.T, kQThreads, 0, stream>>>(a);
   if (prof) prof->before(2, stream);
-  gateup_kernel<<<n_sms, kG1Threads, s1, stream>>>(a);
-  requant_kernel<<<n_sms * 4, 96, 0, stream>>>(a);
-  down_kernel<<<n_sms, kG2Threads, s2, stream>>>(a);
+  if (a.tc) {
+    if ((err = launch_prefill_tc(a, n_sms, stream, 0)) != cudaSuccess) return err;
+  } else {
+    gateup_kernel<<<n_sms, kG1Threads, s1, stream>>>(a);
+  }
+  requant_kernel<<<n_sms * 2, 256, 0, stream>>>(a);
+  if (a.tc) {
+    if ((err = launch_prefill_tc(a, n_sms, stream, 1)) != cudaSuccess) return err;
+  } else {
+    down_kernel<<<n_sms, kG2Threads, s2, stream>>>(a);
+  }
   if (prof) prof->after(stream);
   if (a.dbg.h || a.dbg.qh || a.dbg.sh) debug_kernel<<<n_sms * 4, 256, 0, stream>>>(a);
   finalize_kernel<<<n_sms * 4, 256, 0, stream>>>(a);

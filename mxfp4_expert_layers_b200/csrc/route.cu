@@ -228,6 +228,106 @@ route_kernel(RouteArgs a) {
   MOE_TRACE_POINT(0, 6);
 }
 
+// ---------------------------------------------------------------------
+// Many tokens (T > kRouteGemmMinTokens): the logits as a GEMM on the FP64
+// tensor-core path (mma.sync m8n8k4 f64), then one CTA per token for the
+// top-k.  Every bf16 x bf16 product is exact in float64 and is added with
+// float64 rounding, as in route_kernel (only the order of the additions
+// differs).
+constexpr int kRgTile = 32;  // tokens and experts per CTA
+constexpr int kRgK = 64;     // K per shared-memory stage
+constexpr int kRgLd = kRgK + 4;  // row stride (doubles): 2 wavefronts per fragment load
+
+__device__ __forceinline__ void dmma(double (&d)[2], double a0, double b0) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a0), "d"(b0));
+}
+
+// grid (ceil(E / 32), ceil(T / 32)), 128 threads: warp (wm, wn) computes
+// tokens wm*16 .. +15 x experts wn*16 .. +15 of the CTA's tile as 2 x 2
+// 8 x 8 tiles.  Fragments (m8n8k4, f64): A[r][c] at lane 4r + c, B[c][n] at
+// lane 4n + c, C[r][2c + i] at lane 4r + c.
+__global__ void __launch_bounds__(128) route_gemm_kernel(RouteArgs a) {
+  __shared__ double xs[kRgTile][kRgLd];
+  __shared__ double ws[kRgTile][kRgLd];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 1, wn = warp & 1;
+  const int e0 = blockIdx.x * kRgTile, t0 = blockIdx.y * kRgTile;
+  const int H = a.H;
+  double acc[2][2][2] = {};
+  // staging: thread -> row tid / 4 (of x, then of W), 16 consecutive K
+  const int srow = tid >> 2, sk = (tid & 3) * 16;
+  const bool tok_ok = t0 + srow < a.T, exp_ok = e0 + srow < a.E;
+  const uint4* xrow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(tok_ok ? t0 + srow : 0) * H);
+  const uint4* wrow = reinterpret_cast<const uint4*>(a.Wr + static_cast<size_t>(exp_ok ? e0 + srow : 0) * H);
+  uint4 xv[2], wv[2];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      xv[i] = tok_ok ? __ldcg(xrow + (k0 + sk) / 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+      wv[i] = exp_ok ? __ldg(wrow + (k0 + sk) / 8 + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  load(0);
+  for (int k0 = 0; k0 < H; k0 += kRgK) {
+    __syncthreads();  // the previous stage is consumed
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+      const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = sk + 8 * i + 2 * j;
+        xs[srow][k] = static_cast<double>(__uint_as_float(xw[j] << 16));
+        xs[srow][k + 1] = static_cast<double>(__uint_as_float(xw[j] & 0xFFFF0000u));
+        ws[srow][k] = static_cast<double>(__uint_as_float(ww[j] << 16));
+        ws[srow][k + 1] = static_cast<double>(__uint_as_float(ww[j] & 0xFFFF0000u));
+      }
+    }
+    __syncthreads();
+    if (k0 + kRgK < H) load(k0 + kRgK);  // next stage in flight during the MMAs
+#pragma unroll 4
+    for (int kk = 0; kk < kRgK; kk += 4) {
+      const int c = kk + (lane & 3);
+      const double a0 = xs[wm * 16 + (lane >> 2)][c], a1 = xs[wm * 16 + 8 + (lane >> 2)][c];
+      const double b0 = ws[wn * 16 + (lane >> 2)][c], b1 = ws[wn * 16 + 8 + (lane >> 2)][c];
+      dmma(acc[0][0], a0, b0);
+      dmma(acc[0][1], a0, b1);
+      dmma(acc[1][0], a1, b0);
+      dmma(acc[1][1], a1, b1);
+    }
+  }
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 2; ++ni)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int t = t0 + wm * 16 + mi * 8 + (lane >> 2);
+        const int e = e0 + wn * 16 + ni * 8 + 2 * (lane & 3) + i;
+        if (t < a.T && e < a.E) {
+          float l = static_cast<float>(acc[mi][ni][i]);
+          if (a.bias) l = __fadd_rn(l, a.bias[e]);
+          a.logits[static_cast<size_t>(t) * a.E + e] = l;
+        }
+      }
+}
+
+// One CTA (4 warps) per token: top-k of its logits, weights, and the counts
+// (zeroed before the launch).
+__global__ void __launch_bounds__(kWarps * 32) route_topk_kernel(RouteArgs a) {
+  __shared__ float c_val[kWarps * MOE_MAX_TOPK];
+  __shared__ int c_id[kWarps * MOE_MAX_TOPK];
+  const int t = blockIdx.x;
+  cta_topk(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, a.ids + static_cast<size_t>(t) * a.k,
+           a.w + static_cast<size_t>(t) * a.k, c_val, c_id);
+  if (a.counts && threadIdx.x < a.k) {
+    const int id = a.ids[static_cast<size_t>(t) * a.k + threadIdx.x];
+    atomicAdd(a.counts + id, 1);
+  }
+}
+
 }  // namespace
 
 #ifdef MOE_TRACE
@@ -237,6 +337,15 @@ extern "C" int moe_trace_read_route(unsigned long long* out) {
 #endif
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
+  if (a.T > kRouteGemmMinTokens) {
+    cudaError_t err = cudaSuccess;
+    if (a.counts && (err = cudaMemsetAsync(a.counts, 0, static_cast<size_t>(a.E) * sizeof(int32_t), stream)) !=
+                        cudaSuccess)
+      return err;
+    route_gemm_kernel<<<dim3((a.E + kRgTile - 1) / kRgTile, (a.T + kRgTile - 1) / kRgTile), 128, 0, stream>>>(a);
+    route_topk_kernel<<<a.T, kWarps * 32, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
   dim3 grid((a.E + kWarps - 1) / kWarps, (a.T + kTokTile - 1) / kTokTile);
   RouteArgs args = a;
   void* kargs[] = {&args};
