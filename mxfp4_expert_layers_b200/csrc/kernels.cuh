@@ -1,6 +1,7 @@
 // Launch functions of the MoE kernels (host side).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -124,21 +125,29 @@ struct PrefillArgs {
   float* yacc32;            // [T][H] float32 accumulator of the tcgen05 kernels (same memory), zero between calls
   int* err;
   moe_debug dbg;
+  // TMA tensor maps of the packed weights for the tcgen05 kernels (one
+  // K chunk of 8 consecutive tiles per copy): codes and scales of w13, w2
+  CUtensorMap tm13c, tm13s, tm2c, tm2s;
 };
 
 // Byte offset of code k (fragment order) of panel row R: K is cut into
-// chunks of 256 codes; a chunk holds the rows in bands of 8, each band 16
-// pieces of 8 rows x 16 codes (the no-swizzle K-major layout of tcgen05
-// operands, 2048 bytes per band).
+// chunks of kPanelChunk codes; a chunk holds the rows in bands of 8, each
+// band kPanelChunk/16 pieces of 8 rows x 16 codes (the no-swizzle K-major
+// layout of tcgen05 operands, kPanelBand bytes per band).
+constexpr int kPanelChunk = 128;
+constexpr int kPanelBand = 8 * kPanelChunk;
 __host__ __device__ inline size_t panel_off(int R, int k, int rcap) {
-  return static_cast<size_t>(k >> 8) * (static_cast<size_t>(rcap >> 3) * 2048) +
-         static_cast<size_t>(R >> 3) * 2048 + static_cast<size_t>(((k & 255) >> 4) * 128 + (R & 7) * 16 + (k & 15));
+  return static_cast<size_t>(k / kPanelChunk) * (static_cast<size_t>(rcap >> 3) * kPanelBand) +
+         static_cast<size_t>(R >> 3) * kPanelBand +
+         static_cast<size_t>(((k % kPanelChunk) >> 4) * 128 + (R & 7) * 16 + (k & 15));
 }
 size_t prefill_smem_bytes(int H, int I, int which);
 constexpr int kItemBaseStride = MOE_MAX_EXPERTS + MOE_MAX_SHARED + 1;
 // Grouped GEMMs on tcgen05 (prefill_tc.cu): shapes they take, shared memory,
 // launch of projection `which` (0 gate/up + SwiGLU, 1 down + combine).
 bool prefill_tc_supported(int H, int I);
+// Encode the tensor maps of a.w13 / a.w2 (a.H, a.I, a.E, a.n_shared set).
+bool prefill_tc_maps(PrefillArgs& a);
 size_t prefill_tc_smem_bytes();
 cudaError_t launch_prefill_tc(const PrefillArgs& a, int n_sms, cudaStream_t stream, int which);
 

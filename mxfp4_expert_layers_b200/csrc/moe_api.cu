@@ -13,6 +13,7 @@ struct moe_handle_s {
   int max_tokens;
   int last_path;
   int prefill_kernel;  // MOE_PREFILL_*
+  bool tc_ok;          // the tcgen05 grouped GEMMs can run (shape, tensor maps)
   void* ws;
   size_t ws_bytes;
   // workspace views
@@ -99,9 +100,10 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const size_t P = T * (cfg->top_k + cfg->n_shared);
   const bool many = max_tokens > MOE_GEMV_MAX_TOKENS;
   // operand panels of the tcgen05 kernels: rows = pairs with every expert's
-  // count rounded up to 8; K cut into chunks of 256 codes, 2048 bytes per band
-  const size_t rcap = (P + 7) / 8 * 8 + 8 * NE;
-  const size_t xg_bytes = (H + 255) / 256 * (rcap / 8) * 2048, qg_bytes = (I + 255) / 256 * (rcap / 8) * 2048;
+  // count rounded up to 8; K cut into chunks (panel_off)
+  const size_t rcap = (P + 7) / 8 * 8 + 8 * NE, nch = moe::kPanelChunk;
+  const size_t xg_bytes = (H + nch - 1) / nch * (rcap / 8) * moe::kPanelBand;
+  const size_t qg_bytes = (I + nch - 1) / nch * (rcap / 8) * moe::kPanelBand;
   const size_t pf_sizes[] = {up256(T * H),                   // xq
                              up256(T * 4),                   // xs
                              up256(NE * 4), up256((NE + 1) * 4), up256((NE + 1) * 4),  // counts offsets roff
@@ -177,6 +179,9 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     f.xg = p; p += pf_sizes[i++];
     f.qg = p; p += pf_sizes[i++];
     f.rcap = static_cast<int>(rcap);
+    f.H = cfg->hidden; f.I = cfg->inter; f.E = cfg->n_experts; f.n_shared = cfg->n_shared;
+    f.w13 = weights->w13; f.w2 = weights->w2;
+    h->tc_ok = moe::prefill_tc_supported(cfg->hidden, cfg->inter) && moe::prefill_tc_maps(f);
   }
   *out = h;
   return MOE_OK;
@@ -239,7 +244,7 @@ int prefill_call(moe_handle h, const uint16_t* x, int T, const int32_t* ids, con
   a.x = x; a.ids = ids; a.w = w; a.w13 = h->w.w13; a.w2 = h->w.w2; a.y = y;
   a.err = h->err;
   if (dbg) a.dbg = *dbg;
-  const bool tc = h->prefill_kernel != MOE_PREFILL_EXACT && moe::prefill_tc_supported(c.hidden, c.inter);
+  const bool tc = h->prefill_kernel != MOE_PREFILL_EXACT && h->tc_ok;
   if (h->prefill_kernel == MOE_PREFILL_TCGEN05 && !tc) return MOE_ERR_UNSUPPORTED;
   a.tc = tc ? 1 : 0;
   h->last_path = tc ? 3 : 2;
@@ -296,8 +301,7 @@ int moe_last_path(moe_handle h) { return h ? h->last_path : 0; }
 
 int moe_set_prefill_kernel(moe_handle h, int kind) {
   if (!h || kind < MOE_PREFILL_AUTO || kind > MOE_PREFILL_EXACT) return MOE_ERR_ARG;
-  if (kind == MOE_PREFILL_TCGEN05 && !moe::prefill_tc_supported(h->cfg.hidden, h->cfg.inter))
-    return MOE_ERR_UNSUPPORTED;
+  if (kind == MOE_PREFILL_TCGEN05 && !h->tc_ok) return MOE_ERR_UNSUPPORTED;
   h->prefill_kernel = kind;
   return MOE_OK;
 }
