@@ -50,6 +50,15 @@ def parse():
     return p.parse_args()
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full
+# capture of the current kernels: decode_kernel on a 2-layer stack at T = 1
+# (62.48 MB per launch, scaled per layer: traffic grows with the layers a
+# launch runs), and tc_gemm_kernel<0> + tc_gemm_kernel<1> of one 512-token
+# prefill call (Zipf routing, 103 + 1 experts touched).
+NCU_DECODE_DRAM_BYTES_PER_LAYER = 62.478592e6 / 2
+NCU_PREFILL_GEMM_DRAM_BYTES = 228.321024e6 + 11.817728e6 + 116.868352e6 + 3.162112e6
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -352,7 +361,8 @@ def run_ours(args):
     layer_gbs = ab["layer"] / (layer_us * 1e3)
     roof = {"bound": "hbm", "kernel": "decode_kernel", "achieved": L * ab["layer"] / (dk_us * 1e3),
             "peak": hbm_peak, "unit": "GB/s", "peak_kind": f"{peak_kind} copy bandwidth (burst)",
-            "frac": L * ab["layer"] / (dk_us * 1e3) / hbm_peak, "traffic": None,
+            "frac": L * ab["layer"] / (dk_us * 1e3) / hbm_peak,
+            "traffic": (NCU_DECODE_DRAM_BYTES_PER_LAYER * L if T == 1 and args.workload != "stack42" else None),
             "alg_bytes_per_launch": L * ab["layer"], "avg_launch_us": dk_us, "launches_timed": dk_n,
             "layers_per_launch": L}
 
@@ -515,7 +525,8 @@ def run_prefill(args):
                          "achieved": flops / (gemm_us * 1e6),
                          "peak": fp8_peak, "unit": "TFLOP/s",
                          "peak_kind": "measured bf16 cuBLAS burst x 2 (nominal fp8/bf16 ratio)",
-                         "frac": flops / (gemm_us * 1e6) / fp8_peak, "traffic": None,
+                         "frac": flops / (gemm_us * 1e6) / fp8_peak,
+                         "traffic": NCU_PREFILL_GEMM_DRAM_BYTES if tc else None,
                          "hbm_gbs_of_call": bytes_ / (call_us * 1e3), "avg_launch_us": gemm_us},
             "cpu_baseline": None, "gpu_launches": args.steps * 9, "clocks": clk,
             "timing": "CUDA graph of K calls (route + dispatch + grouped GEMMs + combine)"}
