@@ -204,11 +204,28 @@ def oracle_sample(n_tokens: int, T: int = 1, budget_s: float = 20.0):
             "sample": f"{len(times)} call(s) of {T} token(s), E=512 layers, float64 numpy oracle"}
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (x itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_token_value(ms_total: float, steps: int, layers: int, tokens: int, world: int) -> float:
+    """Whole-job µs per token and layer: every rank pushed steps x tokens
+    tokens through the layers within the (max over ranks) time."""
+    return 1e3 * ms_total / (steps * layers) / (tokens * world)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    T = 4 if args.workload == "verify4" else 1
+    T = 4 if args.workload == "verify4" else 8 if args.workload == "prefill512" else 1
     for _ in range(args.warmup):
         oracle_sample(1, T, 1e9)
     t0 = time.perf_counter()
@@ -233,6 +250,8 @@ def workload_config(args, layers):
              "chained by the residual + RMSNorm harness, one persistent launch per token")
     elif args.workload == "verify4":
         w = f"4-token verify call (i.i.d. tokens) through {n} chained E=512 layers, one launch per call"
+    elif args.workload == "prefill512":
+        w = "chunked prefill: 512 tokens per call, E=512 top-8 + 1 shared, Zipf(1.1) bias"
     else:
         w = "42-layer decode stack, Zipf(1.1) router bias, residual + RMSNorm chain, one launch per token"
     c = {"workload": w, "layers_resident": n, "hidden": H, "inter": I, "experts": E, "top_k": K_TOP,
@@ -317,10 +336,7 @@ def run_ours(args):
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
     assert moe.moe_stack_device_error(stack) == moe.MOE_OK
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, "cuda")
 
     # ---- the stack kernel's own duration: events around every launch
     moe.moe_stack_profile_begin(stack, args.steps + 2)
@@ -357,7 +373,7 @@ def run_ours(args):
     if args.workload == "stack42":
         value = step_us / world                      # us per token through the 42-layer stack
     else:
-        value = layer_us / (T * world)               # us per token per layer
+        value = per_token_value(ms, args.steps, L, T, world)
     layer_gbs = ab["layer"] / (layer_us * 1e3)
     roof = {"bound": "hbm", "kernel": "decode_kernel", "achieved": L * ab["layer"] / (dk_us * 1e3),
             "peak": hbm_peak, "unit": "GB/s", "peak_kind": f"{peak_kind} copy bandwidth (burst)",
@@ -490,10 +506,7 @@ def run_prefill(args):
     barrier()
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, "cuda")
     # grouped GEMM kernels alone (gate/up .. down), events around them
     for h in layers.handles:
         moe.moe_profile_begin(h, args.steps + 2)
