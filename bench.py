@@ -42,7 +42,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42", "prefill512"])
+    p.add_argument("--workload", default="layer", choices=["layer", "verify4", "stack42", "prefill512", "lmhead"])
     p.add_argument("--layers", type=int, default=64)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--prefill-kernel", default="auto", choices=["auto", "tcgen05", "exact"],
@@ -394,11 +394,7 @@ def run_ours(args):
         xo.copy_(x, non_blocking=True)
     ev1.record(stream)
     barrier()
-    e2e_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
     e2e_step_us = 1e3 * e2e_ms / args.steps
     e2e_val = (e2e_step_us if args.workload == "stack42" else e2e_step_us / (L * T)) / world
 
@@ -561,6 +557,108 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+def run_lmhead(args):
+    """FP8 output layer, 157,184 x 2,560, one token per call (the decode step's
+    other weight-bound operation): quantised once, then K calls timed."""
+    import torch
+    import torch.distributed as dist
+    import mxfp4_expert_layers_b200 as moe
+    import synth
+    import synth.gpu
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    moe.load()
+    hbm_peak, peak_kind = peaks()
+    V, T = 157184, 1
+    w = torch.empty((V, H), dtype=torch.int16, device="cuda")
+    synth.gpu.fill_lmhead(w, 0, V, H)
+    q = torch.empty((V, H), dtype=torch.uint8, device="cuda")
+    sw = torch.empty((V,), dtype=torch.float32, device="cuda")
+    moe.moe_lmhead_quantize(w, V, H, q, sw)
+    del w
+    nsteps = args.warmup + args.steps
+    xs_host = np.stack([synth.hidden_states(0, 3000 + 7919 * rank + i, T, H) for i in range(min(nsteps, 256))])
+    xs = torch.from_numpy(xs_host.view(np.int16)).cuda()
+    out = torch.empty((T, V), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, s):
+        moe.moe_lmhead_logits(q, sw, V, H, xs[i % xs.shape[0]], T, out, s)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i, stream)
+    barrier()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(args.steps):
+                step(args.warmup + i, cap)
+    g.replay()
+    barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    g.replay()
+    ev1.record(stream)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
+    clk = clocks.stop()
+    # e2e: x from pinned host memory, logits back to pinned host memory, every call
+    xh = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
+    oh = torch.empty((T, V), dtype=torch.float32).pin_memory()
+    xd = torch.empty((T, H), dtype=torch.int16, device="cuda")
+    barrier()
+    ev0.record(stream)
+    for i in range(args.steps):
+        xd.copy_(xh[i % xh.shape[0]], non_blocking=True)
+        moe.moe_lmhead_logits(q, sw, V, H, xd, T, out, stream)
+        oh.copy_(out, non_blocking=True)
+    ev1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), "cuda")
+    call_us = 1e3 * ms / args.steps
+    alg = V * H + V * 4 + T * H * 2 + T * V * 4
+    gbs = alg / (call_us * 1e3)
+    line = {"metric": METRIC, "value": call_us / (T * world), "unit": "us/token (FP8 LM head, 157184 x 2560)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 x e4m3 (mma.sync), f32 accumulation",
+            "data": "synthetic (seeded SplitMix64 weights, Irwin-Hall normals)",
+            "config": {"workload": "FP8 output layer: 157,184 x 2,560 weights quantised per row, 1 token per call",
+                       "l2": "weights 402 MB > L2"},
+            "roofline": {"bound": "hbm", "kernel": "lmhead_gemv_kernel", "achieved": gbs, "peak": hbm_peak,
+                         "unit": "GB/s", "peak_kind": peak_kind + " copy bandwidth (burst)", "frac": gbs / hbm_peak,
+                         "traffic": None, "alg_bytes_per_launch": alg, "avg_launch_us": call_us,
+                         "frac_of_8tbs": gbs / 8000.0},
+            "cpu_baseline": None,
+            "e2e": {"value": 1e3 * e2e_ms / args.steps / (T * world), "unit": "us/token (FP8 LM head, 157184 x 2560)",
+                    "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * V * 4},
+            "gpu_launches": args.steps, "clocks": clk,
+            "timing": "CUDA graph of K calls; e2e: eager calls with host copies"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def peaks_bf16():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -575,6 +673,8 @@ def main():
         run_reference(args)
     elif args.workload == "prefill512":
         run_prefill(args)
+    elif args.workload == "lmhead":
+        run_lmhead(args)
     else:
         run_ours(args)
 

@@ -300,6 +300,27 @@ int moe_pack_weights(const moe_config* cfg, const moe_mxfp4_weights* src, int ex
 int moe_quantize_fp8(const float* v, int rows, int cols, uint8_t* q, float* s,
                      cudaStream_t stream);
 
+/* FP8 LM head (the output layer read in full every token; "三项优化是什么？"
+ * item 2 on tanhow.com, "Online FP8 LM head" on aivibenews.ru).
+ *
+ * moe_lmhead_quantize: BF16 weights w [V][H] (device) -> q [V][H] FP8 E4M3
+ * codes and s [V] float32, one scale per row: s = amax/448 (IEEE float32
+ * division, 1 for an all-zero row), q = E4M3(w / s) with round to nearest
+ * even and saturation (the activation quantiser of moe_quantize_fp8).  Run
+ * once when the weights are loaded.
+ *
+ * moe_lmhead_logits: x [T][H] BF16 (device, T = 1..8) -> logits [T][V]
+ * float32:  l[t][v] = s[v] * s_x[t] * sum_k e4m3(q[v][k]) * e4m3(qx[t][k]),
+ * with x quantised per token like the MoE activations (s_x = amax/448).
+ * Products are exact and summed in float32 by the tensor cores.  One
+ * launch; the weights are read once for all T tokens.
+ *
+ * H must be a multiple of 64 (MOE_ERR_SHAPE); pointers 16-byte aligned
+ * (MOE_ERR_ALIGN); null pointers, V < 1 or T outside 1..8: MOE_ERR_ARG. */
+int moe_lmhead_quantize(const uint16_t* w, int V, int H, uint8_t* q, float* s, cudaStream_t stream);
+int moe_lmhead_logits(const uint8_t* q, const float* s, int V, int H, const uint16_t* x, int T,
+                      float* logits, cudaStream_t stream);
+
 /* Harness step for chained layers (not part of the MoE layer):
  * r[t] = bf16(r[t] + y[t]) in place, then
  * x_next[t] = bf16( r[t] / sqrt(mean_k r[t,k]^2 + eps) ).  All [T][H]

@@ -29,7 +29,7 @@ MOE_PREFILL_TCGEN05 = 1
 MOE_PREFILL_EXACT = 2
 
 EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_last_path",
-           "moe_set_prefill_kernel",
+           "moe_set_prefill_kernel", "moe_lmhead_quantize", "moe_lmhead_logits",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
            "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static",
            "moe_decode", "moe_stack_create", "moe_stack_decode", "moe_stack_device_error",
@@ -91,6 +91,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_device_error.argtypes = [p, p]
     L.moe_last_path.argtypes = [p]
     L.moe_set_prefill_kernel.argtypes = [p, i]
+    L.moe_lmhead_quantize.argtypes = [p, i, i, p, p, p]
+    L.moe_lmhead_logits.argtypes = [p, p, i, i, p, i, p, p]
     L.moe_destroy.argtypes = [p]
     L.moe_stack_create.argtypes = [p, i, p]
     L.moe_stack_decode.argtypes = [p, p, p, i, ctypes.c_float, p, p, p, p]
@@ -209,6 +211,17 @@ def moe_device_error(handle: int, stream=None) -> int:
 
 def moe_last_path(handle: int) -> int:
     return load().moe_last_path(handle)
+
+
+def moe_lmhead_quantize(w, V: int, H: int, q, s, stream=None) -> None:
+    """FP8 output layer: q [V][H] E4M3 codes and s [V] row scales of the BF16 w."""
+    _check(load().moe_lmhead_quantize(_ptr(w), V, H, _ptr(q), _ptr(s), _stream(stream)), "moe_lmhead_quantize")
+
+
+def moe_lmhead_logits(q, s, V: int, H: int, x, T: int, logits, stream=None) -> None:
+    """logits [T][V] float32 of T <= 8 BF16 tokens x [T][H] through the FP8 output layer."""
+    _check(load().moe_lmhead_logits(_ptr(q), _ptr(s), V, H, _ptr(x), T, _ptr(logits), _stream(stream)),
+           "moe_lmhead_logits")
 
 
 def moe_set_prefill_kernel(handle: int, kind: int) -> None:

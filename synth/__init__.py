@@ -45,10 +45,12 @@ W2_SCALES = 4
 HIDDEN = 5
 BIAS_PERM = 6
 NOISE = 7
+LM_HEAD = 8
 
 SCALE_LO = 120   # E8M0 exponent range of the synthetic weights
 SCALE_HI = 124
 ROUTER_SIGMA = 0.02
+LM_HEAD_SIGMA = 0.02
 
 
 def mix64(z: np.ndarray) -> np.ndarray:
@@ -151,6 +153,14 @@ def expert_scales(seed: int, layer: int, expert: int, which: str, rows: int, k: 
     nb = k // 32
     v = random_ints(key, nrows * nb, SCALE_LO, SCALE_HI, row0 * nb)
     return v.astype(np.uint8).reshape(nrows, nb)
+
+
+def lmhead_weight(seed: int, vocab: int, hidden: int, row0: int = 0, nrows: int | None = None) -> np.ndarray:
+    """BF16 bits ``[nrows][H]`` of the output layer ``[vocab][H]``, rows
+    ``row0 ..``, ~N(0, 0.02^2)."""
+    n = vocab - row0 if nrows is None else nrows
+    key = stream_key(seed, 0, LM_HEAD, 0)
+    return normals_bf16(key, n * hidden, LM_HEAD_SIGMA, start=row0 * hidden).reshape(n, hidden)
 
 
 def hidden_states(seed: int, step: int, T: int, hidden: int) -> np.ndarray:

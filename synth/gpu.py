@@ -6,7 +6,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-from . import ROUTER_SIGMA, ROUTER_W, SCALE_HI, SCALE_LO, W13_CODES, W13_SCALES, W2_CODES, W2_SCALES
+from . import (LM_HEAD, LM_HEAD_SIGMA, ROUTER_SIGMA, ROUTER_W, SCALE_HI, SCALE_LO, W13_CODES, W13_SCALES,
+               W2_CODES, W2_SCALES)
 
 _LIB = None
 
@@ -53,3 +54,10 @@ def fill_layer(bufs: dict, seed: int, layer: int, n_experts: int, hidden: int, i
                                      H * I // 2, stream))
     _check(L.synth_fill_expert_ints(bufs["w2_scales"].data_ptr(), seed, layer, W2_SCALES, 0, n,
                                     H * I // 32, SCALE_LO, SCALE_HI, stream))
+
+
+def fill_lmhead(buf, seed: int, vocab: int, hidden: int, stream: int = 0) -> None:
+    """Fill ``buf`` (torch CUDA int16/uint16 [vocab][hidden]) with the output
+    layer of ``synth.lmhead_weight``."""
+    _check(lib().synth_fill_normals_bf16(buf.data_ptr(), seed, 0, LM_HEAD, 0, vocab * hidden, LM_HEAD_SIGMA,
+                                         stream))
