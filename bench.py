@@ -51,12 +51,14 @@ def parse():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full
-# capture of the current kernels: decode_kernel on a 2-layer stack at T = 1
+# capture of each current kernel: decode_kernel on a 2-layer stack at T = 1
 # (62.48 MB per launch, scaled per layer: traffic grows with the layers a
 # launch runs), and tc_gemm_kernel<0> + tc_gemm_kernel<1> of one 512-token
 # prefill call (Zipf routing, 103 + 1 experts touched).
 NCU_DECODE_DRAM_BYTES_PER_LAYER = 62.478592e6 / 2
 NCU_PREFILL_GEMM_DRAM_BYTES = 228.321024e6 + 11.817728e6 + 116.868352e6 + 3.162112e6
+# lmhead_gemv_kernel, one 157,184 x 2,560 call (T = 1)
+NCU_LMHEAD_DRAM_BYTES = 403.072768e6 + 3.427328e6
 
 
 def peaks():
@@ -645,7 +647,7 @@ def run_lmhead(args):
                        "l2": "weights 402 MB > L2"},
             "roofline": {"bound": "hbm", "kernel": "lmhead_gemv_kernel", "achieved": gbs, "peak": hbm_peak,
                          "unit": "GB/s", "peak_kind": peak_kind + " copy bandwidth (burst)", "frac": gbs / hbm_peak,
-                         "traffic": None, "alg_bytes_per_launch": alg, "avg_launch_us": call_us,
+                         "traffic": NCU_LMHEAD_DRAM_BYTES, "alg_bytes_per_launch": alg, "avg_launch_us": call_us,
                          "frac_of_8tbs": gbs / 8000.0},
             "cpu_baseline": None,
             "e2e": {"value": 1e3 * e2e_ms / args.steps / (T * world), "unit": "us/token (FP8 LM head, 157184 x 2560)",
