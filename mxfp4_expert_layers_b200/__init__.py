@@ -185,8 +185,9 @@ def moe_forward(handle: int, x, T: int, topk_ids, topk_w, y, dbg: dict | None = 
 
 def moe_decode(handle: int, x, T: int, topk_ids, topk_w, y, expert_counts=None,
                dbg: dict | None = None, stream=None) -> None:
-    """moe_route + moe_forward in one launch (T <= MOE_GEMV_MAX_TOKENS);
-    topk_ids, topk_w and expert_counts are outputs."""
+    """Routing and experts of T tokens: one fused launch for T <= MOE_GEMV_MAX_TOKENS,
+    else moe_route followed by the many-token kernels; topk_ids, topk_w and
+    expert_counts are outputs."""
     d = None
     if dbg:
         d = ctypes.byref(moe_debug(*[_ptr(dbg.get(f)) for f, _ in moe_debug._fields_]))
