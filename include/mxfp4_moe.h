@@ -140,23 +140,26 @@ int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* 
  * T <= MOE_GEMV_MAX_TOKENS runs the fused decode kernel (one launch: FP8
  * quantisation of x, gate/up + SwiGLU, FP8 re-quantisation of h, down and
  * the weighted combine with the shared experts); larger T runs the dispatch +
- * grouped-GEMM path.  Ids outside 0..E-1 are skipped and recorded (see
+ * grouped-GEMM path (tcgen05 or mma.sync kernels, see moe_set_prefill_kernel).
+ * Ids outside 0..E-1 are skipped and recorded (see
  * moe_device_error).  Errors: MOE_ERR_ARG, MOE_ERR_UNSUPPORTED. */
 int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
                 const float* topk_w, uint16_t* y, const moe_debug* dbg,
                 cudaStream_t stream);
 
-/* moe_route followed by moe_forward in ONE kernel launch, for decode and
- * speculative verification (T in 1..MOE_GEMV_MAX_TOKENS): the same ids,
- * weights, counts and y as the two calls (the routing step of "Ling 3.0 是什么"
- * on the tanhow.com page -- 8 of 512 routed experts plus the shared one --
- * followed by the experts).  topk_ids/topk_w [T][top_k] and expert_counts [E]
- * (may be NULL) are written; the other arguments as for moe_forward.
- * Requires the whole grid (one CTA per SM) to be resident at once: a launch
- * that shares the GPU with long-running kernels on other streams waits for
- * them, and gives up with MOE_ERR_TIMEOUT (moe_device_error) after a second.
- * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED (T above
- * MOE_GEMV_MAX_TOKENS or shapes whose tiles do not fit in shared memory). */
+/* moe_route followed by moe_forward: the same ids, weights, counts and y as
+ * the two calls (the routing step of "Ling 3.0 是什么" on the tanhow.com page
+ * -- 8 of 512 routed experts plus the shared one -- followed by the experts).
+ * For decode and speculative verification (T in 1..MOE_GEMV_MAX_TOKENS) it is
+ * ONE kernel launch; larger T (up to the handle's max_tokens) runs moe_route
+ * and then the many-token kernels.  topk_ids/topk_w [T][top_k] and
+ * expert_counts [E] (may be NULL) are written; the other arguments as for
+ * moe_forward.  The single launch requires the whole grid (one CTA per SM)
+ * to be resident at once: a launch that shares the GPU with long-running
+ * kernels on other streams waits for them, and gives up with
+ * MOE_ERR_TIMEOUT (moe_device_error) after a second.
+ * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED (shapes whose
+ * tiles do not fit in shared memory). */
 int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
                int32_t* expert_counts, uint16_t* y, const moe_debug* dbg,
                cudaStream_t stream);
