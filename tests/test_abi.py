@@ -82,3 +82,31 @@ def test_calls_on_null_handle_fail_cleanly():
     assert ei.value.code == moe.MOE_ERR_ARG
     moe.moe_destroy(None)
     assert moe.moe_last_path(None) == 0
+
+
+def test_prefill_kernel_selection_needs_a_handle():
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_set_prefill_kernel(None, moe.MOE_PREFILL_AUTO)
+    assert ei.value.code == moe.MOE_ERR_ARG
+
+
+@pytest.mark.parametrize("V,H,T,ptr,code", [
+    (16, 128, 0, 0x1000, moe.MOE_ERR_ARG),       # no tokens
+    (16, 128, 9, 0x1000, moe.MOE_ERR_ARG),       # more than 8 tokens
+    (0, 128, 1, 0x1000, moe.MOE_ERR_ARG),        # empty vocabulary
+    (16, 96, 1, 0x1000, moe.MOE_ERR_SHAPE),      # H not a multiple of 64
+    (16, 128, 1, 0x1008, moe.MOE_ERR_ALIGN),     # misaligned (never dereferenced)
+])
+def test_lmhead_logits_validates_arguments(V, H, T, ptr, code):
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_lmhead_logits(ptr, ptr, V, H, ptr, T, ptr)
+    assert ei.value.code == code
+
+
+def test_lmhead_quantize_validates_arguments():
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_lmhead_quantize(None, 16, 128, 0x1000, 0x1000)
+    assert ei.value.code == moe.MOE_ERR_ARG
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_lmhead_quantize(0x1000, 16, 100, 0x1000, 0x1000)
+    assert ei.value.code == moe.MOE_ERR_SHAPE
