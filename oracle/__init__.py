@@ -1,6 +1,9 @@
 """CPU oracle for the MXFP4 MoE decode layer -- TEST INFRASTRUCTURE ONLY.
 
-Plain, slow, float64 numpy code that states what the layer computes.  Only
+Plain, slow, float64 code that states what the layer computes, twice: numpy
+(``formats.py``, ``moe.py``, ``lmhead.py``) and plain C++17 with OpenMP over
+matrix rows (``moe_oracle.cpp``, loaded through ``cpp.py``; bit-equal to the
+numpy layer on seeded inputs, and the one timed as the CPU baseline).  Only
 ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
 may import it; the product path (the CUDA library and its Python binding)
 never does, and this package imports nothing from the product.

@@ -74,3 +74,36 @@ def test_tokens_are_independent():
     for t in range(3):
         assert np.array_equal(all3[t], LH.lmhead_logits(q, s, x[t:t + 1])[0])
     assert np.all(LH.lmhead_abs_sum(q, s, x) >= np.abs(all3))
+
+
+def test_abs_sum_exact_rational():
+    """lmhead_abs_sum against an exact rational evaluation of its definition,
+    s_w[v] * s_x[t] * sum_k |e4m3(q_w[v,k]) * e4m3(q_x[t,k])|, with the E4M3
+    values decoded from the OCP OFP8 bit fields, on a shape with V != T so a
+    transposed product cannot pass."""
+    w = synth.lmhead_weight(6, 5, 64)
+    x = synth.hidden_states(6, 4, 3, 64)
+    q, s = LH.lmhead_quantize(w)
+    got = LH.lmhead_abs_sum(q, s, x)
+    assert got.shape == (3, 5)
+    qx, sx = LH.quantize_fp8(OF.bf16_to_f64(x).astype(np.float32))
+    for t in range(3):
+        for v in range(5):
+            acc = sum(abs(_e4m3_fraction(int(q[v, k])) * _e4m3_fraction(int(qx[t, k]))) for k in range(64))
+            ref = acc * Fraction(float(s[v])) * Fraction(float(sx[t]))
+            assert ref > 0
+            assert abs(got[t, v] - float(ref)) <= 1e-15 * float(ref)
+
+
+def test_abs_sum_equals_logits_when_every_product_is_nonnegative():
+    """With non-negative weights and activations no product is negative, so
+    the sum of magnitudes is the logit itself; flipping the sign of one
+    weight row leaves the magnitude sum unchanged and negates the logit."""
+    w = _bf16(np.abs(OF.bf16_to_f64(synth.lmhead_weight(7, 4, 64))).astype(np.float32))
+    x = _bf16(np.abs(OF.bf16_to_f64(synth.hidden_states(7, 3, 2, 64))).astype(np.float32))
+    q, s = LH.lmhead_quantize(w)
+    assert np.array_equal(LH.lmhead_abs_sum(q, s, x), LH.lmhead_logits(q, s, x))
+    wn = _bf16(-OF.bf16_to_f64(w).astype(np.float32))
+    qn, sn = LH.lmhead_quantize(wn)
+    assert np.array_equal(LH.lmhead_abs_sum(qn, sn, x), LH.lmhead_abs_sum(q, s, x))
+    assert np.array_equal(LH.lmhead_logits(qn, sn, x), -LH.lmhead_logits(q, s, x))

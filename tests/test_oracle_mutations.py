@@ -6,8 +6,11 @@ import pytest
 from oracle import formats as F
 from oracle import moe as M
 
+from oracle import lmhead as LHM
+
 import test_oracle_formats as TF
 import test_oracle_layer as TL
+import test_oracle_lmhead as TLH
 
 PINS = [
     TF.test_e2m1_table_matches_ocp,
@@ -25,6 +28,8 @@ PINS = [
     TL.test_matvec_brute_force_rational,
     TL.test_swiglu_matches_torch_silu,
     lambda: TL.test_layer_brute_force_tiny(False),
+    TLH.test_abs_sum_exact_rational,
+    TLH.test_abs_sum_equals_logits_when_every_product_is_nonnegative,
 ]
 
 
@@ -91,6 +96,20 @@ def _matvec_no_scale(packed, scales, q, s):
     return W @ F.e4m3_value(q)
 
 
+def _abs_sum_signed(q_w, s_w, x_bf16):
+    # the magnitude sum with the absolute value dropped: the signed logit
+    return LHM.lmhead_logits(q_w, s_w, x_bf16)
+
+
+def _abs_sum_no_weight_scale(q_w, s_w, x_bf16):
+    return LHM.__dict__["_orig_lmhead_abs_sum"](q_w, np.ones_like(s_w), x_bf16)
+
+
+def _abs_sum_abs_outside(q_w, s_w, x_bf16):
+    # |sum| instead of sum of |products|
+    return np.abs(LHM.lmhead_logits(q_w, s_w, x_bf16))
+
+
 MUTATIONS = {
     "nibble order swapped": [(F, "unpack_e2m1", _swapped_unpack)],
     "gate and up swapped": [(M, "swiglu", _swiglu_swapped)],
@@ -102,6 +121,9 @@ MUTATIONS = {
                              (M, "f64_to_bf16", _bf16_double_rounding)],
     "shared expert weight 0.5": [(M, "moe_forward", _forward_shared_half)],
     "activation scale dropped": [(M, "mxfp4_matvec", _matvec_no_scale)],
+    "LM-head magnitude sum without abs": [(LHM, "lmhead_abs_sum", _abs_sum_signed)],
+    "LM-head magnitude sum without the row scale": [(LHM, "lmhead_abs_sum", _abs_sum_no_weight_scale)],
+    "LM-head magnitude sum as |sum|": [(LHM, "lmhead_abs_sum", _abs_sum_abs_outside)],
 }
 
 
@@ -110,6 +132,7 @@ def test_pins_catch_mutation(name, monkeypatch):
     F._orig_e4m3_encode = F.e4m3_encode
     F._orig_f64_to_bf16 = F.f64_to_bf16
     M._orig_moe_forward = M.moe_forward
+    LHM._orig_lmhead_abs_sum = LHM.lmhead_abs_sum
     for mod, attr, fn in MUTATIONS[name]:
         monkeypatch.setattr(mod, attr, fn)
     caught = []
