@@ -119,14 +119,18 @@ typedef struct {
   float* sh;
 } moe_debug;
 
-/* Create a handle for one layer.  Validates the configuration (MOE_ERR_SHAPE)
+/* Create a handle for one layer (one MoE layer of the tanhow.com page,
+ * section "Ling 3.0 是什么": 8 of 512 routed experts plus 1 shared expert,
+ * MXFP4 weights).  Validates the configuration (MOE_ERR_SHAPE)
  * and pointer alignment (MOE_ERR_ALIGN), then allocates a workspace sized for
  * max_tokens tokens per call (MOE_ERR_CUDA if that fails).  The weights are
  * borrowed, not copied.  *out is set only on success. */
 int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens,
                moe_handle* out);
 
-/* Route T tokens: x [T][H] bfloat16 (device) -> topk_ids [T][top_k] int32
+/* Route T tokens (the routing step of tanhow.com, "Ling 3.0 是什么": each
+ * token picks top_k of the routed experts): x [T][H] bfloat16 (device) ->
+ * topk_ids [T][top_k] int32
  * (descending logit, ties to the lower expert index), topk_w [T][top_k]
  * float32 (renormalised softmax weights, sum 1), expert_counts [E] int32
  * (tokens per routed expert; may be NULL).  One kernel launch.
@@ -134,7 +138,10 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
 int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
               int32_t* expert_counts, cudaStream_t stream);
 
-/* Run the experts of T tokens and combine: x [T][H] bfloat16 (device), the
+/* Run the experts of T tokens and combine (the W4A8 expert step of
+ * tanhow.com, "为什么 DGX Spark 上的 MoE 解码是内存受限的？": MXFP4 weights
+ * against FP8 activations; plus the shared expert of "Ling 3.0 是什么"):
+ * x [T][H] bfloat16 (device), the
  * routing from moe_route (or any ids in 0..E-1 and weights the caller
  * chooses), y [T][H] bfloat16 (device, written).  dbg may be NULL.
  * T <= MOE_GEMV_MAX_TOKENS runs the fused decode kernel (one launch: FP8
@@ -170,9 +177,10 @@ int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float*
  * pool, or a plugin that may not call cudaMalloc (which can also block the
  * device) -- and so cannot call moe_create, which allocates a workspace.
  * The experts run exactly as in moe_forward (same kernel and results), with
- * their scratch memory (SwiGLU outputs, per-expert amax, counters, float64
- * row accumulators: about 690 KB) in one fixed array inside this library,
- * which every GPU that loads the library keeps until the process exits.
+ * their scratch memory (SwiGLU outputs, per-expert amax, counters, the
+ * launch counter and tagged logits: about 575 KB) in one fixed array inside
+ * this library, which every GPU that loads the library keeps until the
+ * process exits.
  *   - Limits: T in 1..MOE_GEMV_MAX_TOKENS, inter <= 1024 and hidden <= 4096;
  *     anything larger returns MOE_ERR_UNSUPPORTED.  Other arguments as for moe_forward
  *     (cfg/weights as for moe_create; packed weights), no debug outputs.
@@ -180,14 +188,26 @@ int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float*
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before capturing a stream into a graph.
  *   - Every call on a device shares the one array: calls that overlap on the
- *     GPU (other streams, other threads) race and give wrong results.  Each
- *     call clears the parts that must start at zero (cudaMemsetAsync on the
- *     stream) before its kernels.
+ *     GPU (other streams, other threads) race and give wrong results.  The
+ *     first call clears the parts that must start at zero; every call that
+ *     completes leaves them zero again, so a call issues only its kernel.
+ *   - Device-side errors (an expert id outside 0..E-1, skipped; a bounded
+ *     wait that gave up) are kept in the array and reported by
+ *     moe_forward_static_device_error, which must be called after an error
+ *     before the next moe_forward_static on that device.
  * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED,
  * MOE_ERR_CUDA. */
 int moe_forward_static(const moe_config* cfg, const moe_weights* weights, const uint16_t* x, int T,
                        const int32_t* topk_ids, const float* topk_w, uint16_t* y,
                        cudaStream_t stream);
+
+/* Synchronise the stream and report (then clear) the device-side errors of
+ * earlier moe_forward_static calls on the current device, as
+ * moe_device_error does for a handle: MOE_ERR_DEVICE for out-of-range expert
+ * ids, MOE_ERR_TIMEOUT if a bounded wait inside the kernel gave up.  After
+ * an error it also clears the array's counters and accumulators.  Allocates
+ * nothing.  Errors: MOE_ERR_CUDA. */
+int moe_forward_static_device_error(cudaStream_t stream);
 
 /* A chained stack of layers run by ONE persistent launch per call (decode
  * of a whole model's MoE layers for 1..MOE_GEMV_MAX_TOKENS tokens).  The
@@ -323,6 +343,39 @@ int moe_quantize_fp8(const float* v, int rows, int cols, uint8_t* q, float* s,
 int moe_lmhead_quantize(const uint16_t* w, int V, int H, uint8_t* q, float* s, cudaStream_t stream);
 int moe_lmhead_logits(const uint8_t* q, const float* s, int V, int H, const uint16_t* x, int T,
                       float* logits, cudaStream_t stream);
+
+/* Expert parallelism: one layer's routed experts split over several GPUs.
+ * The pages run the layer on one device; the layer shards naturally by
+ * expert (each token uses 8 of 512 routed experts, tanhow.com "Ling 3.0
+ * 是什么"), so a GPU can hold a contiguous range of the routed experts and
+ * compute their part of y, with the router replicated and the parts summed
+ * across GPUs (NCCL all-reduce or any other sum) before the one BF16
+ * rounding.
+ *
+ * moe_create_ep: a handle for routed experts expert_lo .. expert_hi-1 of a
+ * layer with cfg->n_experts routed experts.  local->w13 / local->w2 hold the
+ * packed tiles of those experts ([expert_hi - expert_lo][...], same tile
+ * layout as moe_weights), followed by the n_shared shared experts when
+ * with_shared is non-zero (one GPU adds them); local->router_w and
+ * router_bias are the whole router [E][H].  max_tokens <= MOE_GEMV_MAX_TOKENS.
+ * moe_forward and moe_decode return MOE_ERR_UNSUPPORTED on such a handle.
+ * Errors: MOE_ERR_ARG (range, max_tokens), those of moe_create.
+ *
+ * moe_decode_partial: routing of T <= MOE_GEMV_MAX_TOKENS tokens (every
+ * GPU computes the same ids, weights and counts, as moe_decode) and this
+ * handle's part of y: y_part [T][H] float32 (device) = sum over the token's
+ * routed experts in the handle's range of w * FFN(x) (+ the shared experts
+ * when the handle adds them), not rounded.  The sum of all parts, rounded
+ * once to BF16 (moe_round_bf16), is moe_decode's y up to the float32
+ * additions of the parts.  One launch.  Errors: MOE_ERR_ARG, MOE_ERR_ALIGN.
+ *
+ * moe_round_bf16: out[i] = BF16 bits of v[i], round to nearest even (n
+ * elements, device pointers).  Errors: MOE_ERR_ARG. */
+int moe_create_ep(const moe_config* cfg, const moe_weights* local, int max_tokens, int expert_lo,
+                  int expert_hi, int with_shared, moe_handle* out);
+int moe_decode_partial(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
+                       int32_t* expert_counts, float* y_part, cudaStream_t stream);
+int moe_round_bf16(const float* v, size_t n, uint16_t* out, cudaStream_t stream);
 
 /* Harness step for chained layers (not part of the MoE layer):
  * r[t] = bf16(r[t] + y[t]) in place, then

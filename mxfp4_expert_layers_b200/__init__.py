@@ -32,6 +32,7 @@ EXPORTS = ("moe_create", "moe_route", "moe_forward", "moe_device_error", "moe_la
            "moe_set_prefill_kernel", "moe_lmhead_quantize", "moe_lmhead_logits",
            "moe_destroy", "moe_strerror", "moe_quantize_fp8", "moe_residual_rmsnorm",
            "moe_profile_begin", "moe_profile_end", "moe_pack_weights", "moe_forward_static",
+           "moe_forward_static_device_error", "moe_create_ep", "moe_decode_partial", "moe_round_bf16",
            "moe_decode", "moe_stack_create", "moe_stack_decode", "moe_stack_device_error",
            "moe_stack_profile_begin", "moe_stack_profile_end", "moe_stack_destroy")
 MOE_PROFILE_KERNELS = 4
@@ -105,6 +106,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.moe_pack_weights.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_mxfp4_weights), i, i,
                                     p, p, p]
     L.moe_forward_static.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), p, i, p, p, p, p]
+    L.moe_forward_static_device_error.argtypes = [p]
+    L.moe_create_ep.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), i, i, i, i,
+                                ctypes.POINTER(p)]
+    L.moe_decode_partial.argtypes = [p, p, i, p, p, p, p, p]
+    L.moe_round_bf16.argtypes = [p, ctypes.c_size_t, p, p]
     L.moe_profile_begin.argtypes = [p, i]
     L.moe_profile_end.argtypes = [p, p, p]
     L.moe_quantize_fp8.argtypes = [p, i, i, p, p, p]
@@ -203,6 +209,36 @@ def moe_forward_static(hidden: int, inter: int, n_experts: int, top_k: int, n_sh
     w = moe_weights(*[_ptr(weights.get(f)) for f, _ in moe_weights._fields_])
     _check(load().moe_forward_static(ctypes.byref(cfg), ctypes.byref(w), _ptr(x), T, _ptr(topk_ids),
                                      _ptr(topk_w), _ptr(y), _stream(stream)), "moe_forward_static")
+
+
+def moe_create_ep(hidden: int, inter: int, n_experts: int, top_k: int, n_shared: int, weights: dict,
+                  max_tokens: int, expert_lo: int, expert_hi: int, with_shared: bool) -> int:
+    """A handle for routed experts expert_lo .. expert_hi-1 of a layer split
+    over GPUs (``weights``: the full router, and w13 / w2 holding those
+    experts' packed tiles, then the shared experts when ``with_shared``)."""
+    cfg = moe_config(hidden, inter, n_experts, top_k, n_shared)
+    w = moe_weights(*[_ptr(weights.get(f)) for f, _ in moe_weights._fields_])
+    h = ctypes.c_void_p()
+    _check(load().moe_create_ep(ctypes.byref(cfg), ctypes.byref(w), max_tokens, expert_lo, expert_hi,
+                                int(bool(with_shared)), ctypes.byref(h)), "moe_create_ep")
+    return h.value
+
+
+def moe_decode_partial(handle: int, x, T: int, topk_ids, topk_w, y_part, expert_counts=None, stream=None) -> None:
+    """Routing of T tokens and this handle's float32 part of y."""
+    _check(load().moe_decode_partial(handle, _ptr(x), T, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_counts),
+                                     _ptr(y_part), _stream(stream)), "moe_decode_partial")
+
+
+def moe_round_bf16(v, n: int, out, stream=None) -> None:
+    """BF16 bits of n float32 values, round to nearest even."""
+    _check(load().moe_round_bf16(_ptr(v), n, _ptr(out), _stream(stream)), "moe_round_bf16")
+
+
+def moe_forward_static_device_error(stream=None) -> int:
+    """Device-side errors of earlier moe_forward_static calls on the current
+    device; returns the code (does not raise)."""
+    return load().moe_forward_static_device_error(_stream(stream))
 
 
 def moe_device_error(handle: int, stream=None) -> int:

@@ -50,6 +50,7 @@ constexpr unsigned long long kWaitNs = 1000ull * 1000 * 1000;
 // Device-side error bits kept in the workspace.
 constexpr int kErrBadId = 1;
 constexpr int kErrTimeout = 2;
+constexpr int kErrRouteBound = 4;  // the many-token router's error bound did not hold
 
 // -------------------------------------------------------------- conversion --
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {

@@ -12,41 +12,55 @@
 // speculative verify step (devotd.net retelling, section 3: verifying four
 // positions touches up to 32 experts).
 //
-// One CTA per SM, 16 warps in 4 groups of 4.  A CTA streams its share of a
-// layer through shared memory with 1-D bulk copies: its slice of router rows
-// (own region, the next layer's rows prefetched as soon as the current ones
-// are used), its gate/up tiles (a ring of NG fixed slots) and its down slabs
-// (a ring of ND slots).  Entry j of a ring lives in slot j mod N; the group
-// that consumes entry j refills the slot with entry j + N, so no thread
-// coordinates the copies.
+// The step reads every weight byte once and is bound by HBM, so the design
+// goal is that every byte a CTA needs is requested as soon as it is known
+// and that nothing serialises the consumption of the bytes that landed.
+//
+// One CTA per SM, 16 warps.  Weights move through ONE ring of NS equal
+// shared-memory slots.  The CTA's work of a layer is a list of entries: its
+// gate/up tiles (8 gate + 8 up rows of one expert, all of K) and then its
+// down slabs (16 output rows of one expert, all of K) packed `dpe` to an
+// entry.  Entry n of the whole launch (numbered across layers) lives in
+// slot n mod NS and is issued (1-D bulk copies completing on the slot's
+// mbarrier) as soon as entry n - NS has been consumed: right after routing
+// the CTA requests min(NS, entries) of them at once; the rest follow as
+// slots free up.
 //
 // Per layer (each CTA):
 //  1. input x: the call's x for the first layer; afterwards
 //     r = bf16(r + y_prev), x = bf16(r / sqrt(mean(r^2) + eps)) from the
 //     previous layer's y (float64, every CTA the same values); FP8 E4M3 codes
 //     of x with one amax/448 scale per token.
-//  2. logits of the CTA's router rows (float64 sums of exact products,
-//     rounded once to float32, plus the bias); a grid-wide arrive/wait; then
-//     every CTA selects the same top-k from the same logits.
-//  3. gate/up: tile i (8 gate + 8 up rows of one expert) belongs to CTA
-//     i mod G; the CTA's tile j goes to warp group j mod 4, whose 4 warps
-//     split its blocks.  One mma.sync m16n8k32 e4m3 per block gives exact
-//     block sums, scaled by 2^(E-127+6) and summed in float64.  The group
-//     reduces the tile, applies SwiGLU in float64 -> h (float32) and raises
-//     the per-(expert, token) amax.  Groups synchronise only among
-//     themselves (named barriers).
+//  2. logits of the CTA's router rows (in shared memory, fetched during the
+//     previous layer; float64 sums of exact products rounded once to
+//     float32, plus the bias), published as 64-bit words tagged with the
+//     launch and layer; every CTA reads all of them until each carries the
+//     current tag (no separate grid barrier), selects the same top-k and
+//     issues its entries.
+//  3. gate/up: tile j of the CTA is split along K into 4 quarters taken by
+//     the 4 warps of group j mod 4; one mma.sync m16n8k32 e4m3 per 32-element
+//     block gives the block sums, scaled by 2^(E-127+6) and summed in
+//     float64.  Each warp leaves its partial sums in shared memory and counts
+//     itself in; the last of the 4 refills the slot and finishes the tile:
+//     SwiGLU in float64 -> h (float32, global) and the per-(expert, token)
+//     amax.  No warp waits for another.
 //  4. down: after a grid-wide arrive/wait, h is re-quantised with amax/448
-//     into shared memory; slab i of the CTA's range of (row tile, expert)
-//     slabs goes to group i mod 4, the routing weight and h scale folded
-//     into the float64 epilogue.  Row tiles the CTA owns are rounded to
-//     bfloat16 directly; a row tile shared with a neighbouring CTA is summed
-//     in a float64 accumulator and rounded by whichever CTA adds last.
-//  5. a grid-wide arrive marks y complete for the next layer.
+//     into shared memory; the CTA's slabs (a contiguous range of the
+//     (row tile, expert) slabs, split along K when there are few) are taken
+//     by the warps round robin and summed, times the routing weight and the
+//     h scale, into float64 row accumulators in shared memory.  Row tiles the
+//     CTA owns are rounded to bfloat16 directly; a row tile shared with a
+//     neighbouring CTA is summed in a float64 accumulator in global memory
+//     and rounded by whichever CTA adds last.  The next layer's shared-expert
+//     tiles are requested as soon as the CTA's slabs are done.
+//  5. a stacked layer's y is published as 64-bit words (two bfloat16 rows |
+//     tag << 32); the next layer reads them as they arrive (no grid barrier).
 //
 // Every wait is bounded (one second of %globaltimer) and records
-// kErrTimeout; a CTA that gave up lets its copies in flight land and exits.
-// The grid must be co-resident (one CTA per SM, G <= SM count); the
-// launcher sizes it so.
+// kErrTimeout; a warp that gives up raises a CTA-wide abort flag, and the CTA
+// lets its copies in flight land before it exits.  The grid must be
+// co-resident (one CTA per SM, G <= SM count); the launcher checks that the
+// occupancy allows it.
 #include <atomic>
 #include <cstdio>
 
@@ -59,47 +73,18 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kGroups = 4;           // warp groups
-constexpr int kGW = kWarps / kGroups;  // warps per group
-constexpr int kMaxNG = 16;           // gate/up slots at most
-constexpr int kMaxND = 32;           // down slots at most
-constexpr int kFeat = 8;             // gate/up features per tile
-constexpr int kBatch = 2;            // blocks whose MMAs are in flight together
+constexpr int kGroups = 4;             // gate/up warp groups
+constexpr int kQuarters = kWarps / kGroups;  // warps per tile (K quarters)
+constexpr int kMaxNS = 16;             // ring slots at most
+constexpr int kFeat = 8;               // gate/up features per tile
+constexpr int kBatch = 4;              // blocks whose MMAs are in flight together
+constexpr int kHLoads = 4;             // float4 of h per thread requested at once
+constexpr int kPartBlocks = 8;         // blocks of a down item (K part of a slab)
 constexpr int kMaxDevices = 64;
 
 __host__ __device__ inline size_t up128(size_t v) { return (v + 127) / 128 * 128; }
 __host__ __device__ inline int gu_entry_bytes(int H) { return 272 * (H / 32); }
 __host__ __device__ inline int dn_entry_bytes(int I) { return 272 * (I / 32); }
-
-// Barrier of one warp group (named barrier 1 + grp) that also ORs a flag
-// over the group: every thread gets the same answer.
-__device__ __forceinline__ bool group_sync_or(int grp, bool v) {
-  int r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.s32 q, %1, 0;\n bar.red.or.pred p, %2, %3, q;\n selp.s32 %0, 1, 0, p;\n}\n"
-      : "=r"(r)
-      : "r"(static_cast<int>(v)), "r"(1 + grp), "r"(kGW * 32)
-      : "memory");
-  return r != 0;
-}
-
-// Wait for use `use` of a ring slot: first until its copy has been issued
-// (uses > use; another warp group may still be consuming the previous use),
-// then for the copy's bytes.  Bounded like every wait.
-__device__ __forceinline__ bool wait_slot(uint64_t* bar, const int* uses, int use, int* err) {
-  const volatile int* u = uses;
-  if (*u <= use) {
-    const unsigned long long t0 = global_ns();
-    for (long long i = 1;; ++i) {
-      if (*u > use) break;
-      if ((i & 255) == 0 && global_ns() - t0 > kWaitNs) {
-        if (err) atomicOr(err, kErrTimeout);
-        return false;
-      }
-    }
-  }
-  return mbar_wait_bounded(bar, use & 1, err);
-}
 
 // order-preserving map of a float32 onto uint32 (0 is never produced by a
 // non-NaN value)
@@ -111,15 +96,52 @@ __device__ __forceinline__ float key_f32(unsigned k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 // Top-k of one token's logits by one warp (E <= 512: 16 values per lane),
 // ties to the lower expert index; softmax over the selected logits in float64.
-__device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int32_t* ids, float* w) {
+// The logits are 64-bit words (float bits | tag << 32) written by every CTA
+// for its router rows; the warp reads them until each carries this layer's
+// tag, so the words themselves are the grid-wide hand-off (a single 64-bit
+// store and load are atomic).  Bounded: false (and kErrTimeout) if some
+// logit never arrives.
+__device__ __noinline__ bool topk_warp(const unsigned long long* lg, unsigned tag, int E, int k, int32_t* ids,
+                                       float* w, int* err, const int* abort) {
   const int lane = threadIdx.x & 31;
   unsigned key[16];
+  unsigned pend = 0;
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
-    const int e = lane + 32 * m;
-    key[m] = e < E ? f32_key(__ldcg(lg + e)) : 0u;
+    key[m] = 0u;
+    if (lane + 32 * m < E) pend |= 1u << m;
+  }
+  const unsigned long long t0 = global_ns();
+  for (long long it = 0;; ++it) {
+    unsigned long long v[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (pend >> m & 1u) v[m] = ld_relaxed_u64(lg + lane + 32 * m);
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if ((pend >> m & 1u) && static_cast<unsigned>(v[m] >> 32) == tag) {
+        key[m] = f32_key(__uint_as_float(static_cast<unsigned>(v[m])));
+        pend &= ~(1u << m);
+      }
+    if (__all_sync(0xffffffffu, pend == 0u)) break;
+    if ((it & 7) == 7) {
+      const bool late = global_ns() - t0 > kWaitNs || it > kSpinLimit || *reinterpret_cast<const volatile int*>(abort);
+      if (__any_sync(0xffffffffu, late)) {
+        if (lane == 0) atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
   }
   unsigned taken = 0;  // bit m: element lane + 32 m already selected
   unsigned bk = 0;
@@ -151,6 +173,7 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int32_t
     ids[lane] = my_id;
     w[lane] = static_cast<float>(z / sum);
   }
+  return true;
 }
 
 // The distinct experts of the call, built by one warp: the shared experts
@@ -158,7 +181,7 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int32_t
 // slot); wsum gets the routing weight of each (expert, token) (1 for shared).
 __device__ __forceinline__ void build_distinct(const int32_t* ids, const float* w, int T, int k, int E,
                                                int n_shared, Distinct& d, double (*wsum)[kMaxTokGemv], int* err,
-                                               bool report) {
+                                               bool report, int lo, int hi) {
   const int lane = threadIdx.x & 31;
   const int n = T * k;  // <= 32
   for (int i = lane; i < kMaxDistinct; i += 32) {
@@ -167,8 +190,9 @@ __device__ __forceinline__ void build_distinct(const int32_t* ids, const float* 
   }
   __syncwarp();
   const int e = lane < n ? ids[lane] : -1;
-  const bool valid = lane < n && e >= 0 && e < E;
-  if (lane < n && !valid && report) atomicOr(err, kErrBadId);
+  const bool in_layer = lane < n && e >= 0 && e < E;
+  const bool valid = in_layer && e >= lo && e < hi;  // routed experts held by this call
+  if (lane < n && !in_layer && report) atomicOr(err, kErrBadId);
   const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
   const int first = __ffs(peers) - 1;
   const unsigned lead = __ballot_sync(0xffffffffu, valid && first == lane);
@@ -202,9 +226,28 @@ __device__ __noinline__ void note_timeout(int line, int layer, int entry) {
 #endif
 }
 
-// CTA owning down slab q: the largest c with floor(c * S / G) <= q.
-__device__ __forceinline__ int slab_owner(int q, int S, int G) { return ((q + 1) * G + S - 1) / S - 1; }
-__device__ __forceinline__ int slab_start(int c, int S, int G) { return c * S / G; }
+// Output row tiles (16 rows of y) of CTA c: whole tiles, R / G each and one
+// more for the last R mod G CTAs.  A CTA owns every expert's slab of its row
+// tiles, so each y row is summed and rounded by one CTA.
+__device__ __forceinline__ int rows_of(int c, int R, int G) { return R / G + (c >= G - R % G ? 1 : 0); }
+__device__ __forceinline__ int row0_of(int c, int R, int G) { return (R / G) * c + max(0, c - (G - R % G)); }
+
+// First gate/up tile of CTA c (c = G: the tile count).  The layer's bytes
+// (gate/up tiles and down slabs) are shared out evenly: a CTA's gate/up
+// quota is what its down slabs leave of an even share, and the tiles are
+// given out in proportion to the quotas (integer arithmetic, so every CTA
+// computes the same boundaries).  A CTA's tiles are consecutive.
+__device__ __forceinline__ int gstart_of(int c, int G, int R, int nd, int ntiles, long long gb, long long db) {
+  const long long W = static_cast<long long>(ntiles) * gb + static_cast<long long>(R) * nd * db;
+  const int base = R / G, extra = R % G;
+  // G x (even share - down bytes), for CTAs with base and base + 1 row tiles
+  const long long qa = max(0LL, W - static_cast<long long>(G) * base * nd * db);
+  const long long qb = max(0LL, W - static_cast<long long>(G) * (base + 1) * nd * db);
+  const int nb = max(0, c - (G - extra));  // CTAs before c with base + 1 row tiles
+  const long long P = static_cast<long long>(c - nb) * qa + static_cast<long long>(nb) * qb;
+  const long long PG = static_cast<long long>(G - extra) * qa + static_cast<long long>(extra) * qb;
+  return PG > 0 ? static_cast<int>((P * ntiles + PG / 2) / PG) : 0;
+}
 
 __device__ __forceinline__ LayerW layer_ptrs(const DecodeArgs& a, int l) {
   if (!a.layers) return a.layer0;
@@ -217,52 +260,146 @@ __device__ __forceinline__ LayerW layer_ptrs(const DecodeArgs& a, int l) {
   return w;
 }
 
-// Shared-memory views and the copy bookkeeping of one CTA.
-struct Smem {
-  uint8_t* gu;        // [NG][gu_entry_bytes]
-  uint8_t* dn;        // [ND][dn_entry_bytes]
-  uint8_t* rr;        // router rows
-  uint64_t* fg;       // [NG] full barriers
-  uint64_t* fd;       // [ND]
-  uint64_t* fr;       // router rows
-  int* ug;            // [NG] copies issued into each slot so far
-  int* ud;            // [ND]
-  int* ur;
+// The weight ring of one CTA.
+struct Ring {
+  uint8_t* base;   // [ns][slot] bytes
+  uint64_t* full;  // [ns] one phase per entry
+  int* iss;        // [ns] entries issued into each slot so far
+  int* arr;        // [ns] items of the slot's current entry finished
+  int ns, slot, dpe;
 };
 
-__device__ __forceinline__ void copy_in(uint8_t* dst, const void* src, int bytes, uint64_t* bar, int* uses) {
-  mbar_expect_tx(bar, static_cast<uint32_t>(bytes));
-  bulk_g2s(dst, src, static_cast<uint32_t>(bytes), bar);
-  atomicAdd(uses, 1);
+// What one layer asks of this CTA (the same values in every thread).
+struct Work {
+  int nd;          // distinct experts of the call
+  int g0, ng;      // gate/up tiles g0 .. g0+ng-1 (tile i: features 8 (i mod I/8) of distinct expert i / (I/8))
+  int r0, nr;      // output row tiles r0 .. r0+nr-1
+  int nq;          // down slabs nr * nd: slab k = row tile r0 + k / nd of distinct expert k mod nd
+  int cnt;         // entries: ng tiles, then ceil(nq / dpe) slab groups
+  int dsplit;      // down items per slab (K parts)
+};
+
+__device__ __forceinline__ Work plan_work(const DecodeArgs& a, int nd, int cta, int G, int dpe) {
+  Work w;
+  const int cpe = a.I / kFeat, R = a.H / 16, ntiles = nd * cpe;
+  w.nd = nd;
+  w.g0 = gstart_of(cta, G, R, nd, ntiles, gu_entry_bytes(a.H), dn_entry_bytes(a.I));
+  w.ng = gstart_of(cta + 1, G, R, nd, ntiles, gu_entry_bytes(a.H), dn_entry_bytes(a.I)) - w.g0;
+  w.r0 = row0_of(cta, R, G);
+  w.nr = rows_of(cta, R, G);
+  w.nq = w.nr * nd;
+  w.cnt = w.ng + (w.nq + dpe - 1) / dpe;
+  // K parts of kPartBlocks blocks: a fixed split, so a slab's float32 partial
+  // sums do not depend on how many tokens or slabs the call has
+  w.dsplit = (a.I / 32 + kPartBlocks - 1) / kPartBlocks;
+  return w;
 }
 
-// Gate/up tile j of the CTA for this layer -> its slot (entry gidx).
-__device__ __forceinline__ void issue_gu(const DecodeArgs& a, const Smem& sm, const LayerW& lw, const int* expert,
-                                         int j, int gidx) {
-  const int cpe = a.I / kFeat, i = blockIdx.x + gridDim.x * j, s = gidx % a.ng_slots;
-  const int bytes = gu_entry_bytes(a.H);
-  copy_in(sm.gu + static_cast<size_t>(s) * bytes, lw.w13 + (static_cast<size_t>(expert[i / cpe]) * cpe + i % cpe) * bytes,
-          bytes, &sm.fg[s], &sm.ug[s]);
+// Position of expert e (routed < E, shared E + s) in the weight arrays: the
+// arrays hold the routed experts ep_lo .. ep_hi-1 (all of them unless the
+// layer is split over several GPUs), then the shared experts.
+__device__ __forceinline__ int weight_index(const DecodeArgs& a, int e) {
+  return e < a.E ? e - a.ep_lo : (a.ep_hi - a.ep_lo) + (e - a.E);
 }
 
-// Down slab q -> its slot (entry didx).
-__device__ __forceinline__ void issue_dn(const DecodeArgs& a, const Smem& sm, const LayerW& lw, const int* expert,
-                                         int nd, int q, int didx) {
-  const int s = didx % a.nd_slots, bytes = dn_entry_bytes(a.I);
-  copy_in(sm.dn + static_cast<size_t>(s) * bytes,
-          lw.w2 + (static_cast<size_t>(expert[q % nd]) * (a.H / 16) + q / nd) * bytes, bytes, &sm.fd[s], &sm.ud[s]);
+// Request entry j of the layer (launch-wide entry gidx) into its slot.
+// `expert` maps distinct-expert positions to expert indices.
+__device__ __forceinline__ void issue_entry(const DecodeArgs& a, const Ring& rg, const LayerW& lw, const int* expert,
+                                            const Work& wk, int j, int gidx) {
+  const int s = gidx % rg.ns;
+  uint8_t* dst = rg.base + static_cast<size_t>(s) * rg.slot;
+  if (j < wk.ng) {
+    const int cpe = a.I / kFeat, i = wk.g0 + j, bytes = gu_entry_bytes(a.H);
+    mbar_expect_tx(&rg.full[s], static_cast<uint32_t>(bytes));
+    bulk_g2s(dst, lw.w13 + (static_cast<size_t>(weight_index(a, expert[i / cpe])) * cpe + i % cpe) * bytes,
+             static_cast<uint32_t>(bytes), &rg.full[s]);
+  } else {
+    const int d = j - wk.ng, ka = d * rg.dpe, n = min(rg.dpe, wk.nq - ka);
+    const int bytes = dn_entry_bytes(a.I);
+    mbar_expect_tx(&rg.full[s], static_cast<uint32_t>(n * bytes));
+    for (int k = ka; k < ka + n; ++k)
+      bulk_g2s(dst + (k - ka) * bytes,
+               lw.w2 + (static_cast<size_t>(weight_index(a, expert[k % wk.nd])) * (a.H / 16) + wk.r0 + k / wk.nd) * bytes,
+               static_cast<uint32_t>(bytes), &rg.full[s]);
+  }
+  atomicAdd(&rg.iss[s], 1);
+}
+
+// Items of entry j (the consumers that must count themselves in before the
+// slot is free again).
+__device__ __forceinline__ int entry_items(const Ring& rg, const Work& wk, int j) {
+  if (j < wk.ng) return kQuarters;
+  const int d = j - wk.ng;
+  return min(rg.dpe, wk.nq - d * rg.dpe) * wk.dsplit;
+}
+
+// Wait until entry gidx has landed in its slot: first until it has been
+// issued (the slot's previous entry consumed), then for its bytes.  Bounded;
+// gives up early when another warp raised the abort flag.
+__device__ __noinline__ bool wait_entry_slow(const Ring& rg, int gidx, int* err, int* abort) {
+  const int s = gidx % rg.ns, use = gidx / rg.ns;
+  const volatile int* is = rg.iss + s;
+  const volatile int* ab = abort;
+  const unsigned long long t0 = global_ns();
+  for (long long i = 1; i < kSpinLimit; ++i) {
+    if (*is <= use) __nanosleep(64);  // not issued yet: the slot's previous entry is in use
+    else if (mbar_try_wait_sleep(&rg.full[s], use & 1, 1000u)) return true;
+    if ((i & 15) == 0) {
+      if (*ab) return false;
+      if (global_ns() - t0 > kWaitNs) break;
+    }
+  }
+  atomicOr(err, kErrTimeout);
+  *reinterpret_cast<volatile int*>(abort) = 1;
+  return false;
+}
+__device__ __forceinline__ bool wait_entry(const Ring& rg, int gidx, int* err, int* abort) {
+  const int s = gidx % rg.ns, use = gidx / rg.ns;
+  if (*reinterpret_cast<const volatile int*>(rg.iss + s) > use && mbar_try_wait(&rg.full[s], use & 1)) return true;
+  return wait_entry_slow(rg, gidx, err, abort);
+}
+
+// 8 bfloat16 y values (chunk u of [T][H]) from the tagged words of a layer's
+// y (two values per 64-bit word, tag in the high half): read until all four
+// words carry `tag`.  Bounded; false (kErrTimeout) when a word never arrives.
+__device__ __forceinline__ bool load_y8(const unsigned long long* ty, int u, unsigned tag, uint4& out, int* err,
+                                        const int* abort) {
+  const unsigned long long* p = ty + 4 * static_cast<size_t>(u);
+  unsigned long long v[4];
+  const unsigned long long t0 = global_ns();
+  for (long long it = 0;; ++it) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = ld_relaxed_u64(p + j);
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ok &= static_cast<unsigned>(v[j] >> 32) == tag;
+    if (ok) break;
+    if ((it & 7) == 7 && (global_ns() - t0 > kWaitNs || it > kSpinLimit ||
+                          *reinterpret_cast<const volatile int*>(abort))) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  out = make_uint4(static_cast<unsigned>(v[0]), static_cast<unsigned>(v[1]), static_cast<unsigned>(v[2]),
+                   static_cast<unsigned>(v[3]));
+  return true;
 }
 
 // Residual add and RMS normalisation of the stack (every CTA, same values):
 // r = bf16(r + y); x = bf16(r / sqrt(mean(r^2) + eps)), float64 arithmetic.
-// rs and xb are [T][H] bfloat16 in shared memory.
-__device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t* y, uint16_t* xb,
-                              double (*red)[kMaxTokGemv], double* den_s) {
+// rs and xb are [T][H] bfloat16 in shared memory; y comes from the tagged
+// words of the previous layer (every CTA's rows, read as they arrive).
+// Returns false when a wait gave up (the caller aborts).
+__device__ bool residual_norm(const DecodeArgs& a, uint16_t* rs, const unsigned long long* ty, unsigned tag,
+                              uint16_t* xb, double (*red)[kMaxTokGemv], double* den_s, int* abort) {
   const int H = a.H, T = a.T, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int upr = H / 8;
   double ss[kMaxTokGemv] = {0.0, 0.0, 0.0, 0.0};
-  for (int u = tid; u < T * upr; u += kThreads) {
-    const uint4 yv = __ldcg(reinterpret_cast<const uint4*>(y) + u);
+  bool good = true;
+  for (int u = tid; u < T * upr && good; u += kThreads) {
+    uint4 yv;
+    good = load_y8(ty, u, tag, yv, a.err, abort);
     const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
     const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
@@ -291,7 +428,10 @@ __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t*
     const double v = warp_sum_f64(ss[tt]);
     if (lane == 0) red[warp][tt] = v;
   }
-  __syncthreads();
+  if (!__syncthreads_and(good)) {
+    if (tid == 0) *reinterpret_cast<volatile int*>(abort) = 1;
+    return false;
+  }
   if (tid < T) {
     double s = 0.0;
     for (int w = 0; w < kWarps; ++w) s += red[w][tid];
@@ -313,21 +453,85 @@ __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t*
     reinterpret_cast<uint4*>(xb)[u] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   __syncthreads();
+  return true;
+}
+
+// The float32 factor of one block sum: 2^(E-127) times the 2^6 the E4M3
+// widening of E2M1 took out (see e4m3_lo), i.e. 2^(E-121), built from the
+// E8M0 byte in one integer multiply-add.  Exact for E <= 248; the E8M0 NaN
+// code 255 is not supported.
+__device__ __forceinline__ float block_scale(uint32_t e8) { return __uint_as_float(e8 * (1u << 23) + (6u << 23)); }
+
+// One warp's share of a 16-row tile over blocks [b0, b1): per block one
+// mma.sync m16n8k32 (A = the E2M1 codes widened to E4M3 bytes holding
+// value * 2^-6, B = the FP8 activations of tokens 0..T-1 as columns) gives
+// the float32 block sums (exact when the 32 products span at most 24 bits),
+// scaled by 2^(E-121) and summed in float32 (fused multiply-adds).  acc: rows
+// g and g+8 of tokens 2*t4 and 2*t4+1 (lane = 4g + t4).  `xbp` points at this
+// lane's activation bytes of block 0 (nullptr: a zero column).
+template <int kT>
+__device__ __forceinline__ void tile_blocks(const uint8_t* st, int nb, int b0, int b1, const uint8_t* xbp,
+                                            float (&acc)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2;
+  const uint8_t* cp = st + 8 * lane;
+  const uint8_t* sp = st + 256 * nb + 2 * g;
+  int b = b0;
+  // whole batches: no per-block bounds
+  for (; b + kBatch <= b1; b += kBatch) {
+    float d[kBatch][4];
+    uint32_t sc[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const uint2 cw = *reinterpret_cast<const uint2*>(cp + 256 * (b + u));
+      sc[u] = *reinterpret_cast<const uint16_t*>(sp + 16 * (b + u));
+      const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+      uint2 q = make_uint2(0u, 0u);
+      if (xbp) q = *reinterpret_cast<const uint2*>(xbp + 32 * (b + u));
+      mma_fp8(d[u], af, q.x, q.y);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const float sa = block_scale(sc[u] & 0xFFu), sb = block_scale(sc[u] >> 8);
+      acc[0] = fmaf(d[u][0], sa, acc[0]);
+      acc[2] = fmaf(d[u][2], sb, acc[2]);
+      if (kT > 1) {
+        acc[1] = fmaf(d[u][1], sa, acc[1]);
+        acc[3] = fmaf(d[u][3], sb, acc[3]);
+      }
+    }
+  }
+  // the remaining blocks one at a time
+  for (; b < b1; ++b) {
+    float d[4];
+    const uint2 cw = *reinterpret_cast<const uint2*>(cp + 256 * b);
+    const uint32_t sc = *reinterpret_cast<const uint16_t*>(sp + 16 * b);
+    const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+    uint2 q = make_uint2(0u, 0u);
+    if (xbp) q = *reinterpret_cast<const uint2*>(xbp + 32 * b);
+    mma_fp8(d, af, q.x, q.y);
+    const float sa = block_scale(sc & 0xFFu), sb = block_scale(sc >> 8);
+    acc[0] = fmaf(d[0], sa, acc[0]);
+    acc[2] = fmaf(d[2], sb, acc[2]);
+    if (kT > 1) {
+      acc[1] = fmaf(d[1], sa, acc[1]);
+      acc[3] = fmaf(d[3], sb, acc[3]);
+    }
+  }
 }
 
 // kStack: chained layers with the residual + RMS normalisation between them;
-// kDebug: the optional debug outputs are written.  Four instances keep the
-// code of the common case small (it runs once per layer and its instruction
-// footprint matters).
-template <bool kStack, bool kDebug>
+// kDebug: the optional debug outputs are written; kT1: one token (the
+// common decode case: half the float64 accumulation work).
+template <bool kStack, bool kDebug, bool kT1>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t fg[kMaxNG];
-  __shared__ __align__(8) uint64_t fd[kMaxND];
+  __shared__ __align__(8) uint64_t full[kMaxNS];
   __shared__ __align__(8) uint64_t fr;
-  __shared__ int ug[kMaxNG], ud[kMaxND], ur;
+  __shared__ int iss[kMaxNS], arr[kMaxNS];
+  __shared__ int s_riss;  // router-row copies issued
   __shared__ Distinct dist;
+  __shared__ int s_pre_expert[MOE_MAX_SHARED];
   __shared__ double wsum[kMaxDistinct][kMaxTokGemv];
   __shared__ double coef[kMaxDistinct][kMaxTokGemv];
   __shared__ float shs[kMaxDistinct][kMaxTokGemv];
@@ -342,57 +546,69 @@ decode_kernel(DecodeArgs a) {
   __shared__ double den_s[kMaxTokGemv];
   __shared__ int s_abort;
   __shared__ int s_flag;
-  __shared__ int s_last[2];
   __shared__ int s_hist[MOE_MAX_EXPERTS];
 
-  const int H = a.H, I = a.I, T = a.T, E = a.E, S = a.n_shared, L = a.L;
-  const int NG = a.ng_slots, ND = a.nd_slots;
+  constexpr int kTc = kT1 ? 1 : 2;  // accumulator columns per lane
+  const int H = a.H, I = a.I, T = kT1 ? 1 : a.T, E = a.E, S = a.n_shared, L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = warp / kGW, wg = warp % kGW;
+  const int grp = warp / kQuarters, wq = warp % kQuarters;
   const int G = gridDim.x, cta = blockIdx.x;
   const int cpe = I / kFeat;
+  const int nb = H / 32, nbI = I / 32;
   constexpr bool stack = kStack;
-  const Smem sm{smem, smem + a.dn_off, smem + a.rr_off, fg, fd, &fr, ug, ud, &ur};
+  const Ring rg{smem, full, iss, arr, a.ns, a.slot_bytes, a.dpe};
+  uint8_t* rr = smem + a.rr_off;                                   // router rows
   uint8_t* xq = smem + a.xq_off;                                   // [T][H] permuted E4M3
-  double* redd = reinterpret_cast<double*>(smem + a.red_off);      // group partial sums
-  uint16_t* xb = reinterpret_cast<uint16_t*>(smem + a.red_off);    // [T][H] bf16 x (layer start)
-  uint8_t* qh = smem + a.qh_off;                                   // [pair][I] permuted E4M3
-  double* yg = reinterpret_cast<double*>(smem + a.yrow_off);       // [group][row tile][16][T]
   uint16_t* rs = reinterpret_cast<uint16_t*>(smem + a.rs_off);     // [T][H] bf16 residual (stack)
-  const int yg_len = a.yrow_len;                                   // per group
+  uint16_t* xb = reinterpret_cast<uint16_t*>(smem + a.u_off);      // [T][H] bf16 x (layer start)
+  double* lpart = reinterpret_cast<double*>(smem + a.u_off + a.lpart_off);  // router partial sums
+  float* redp = reinterpret_cast<float*>(smem + a.u_off);          // [ns][4][16][T] gate/up partials
+  uint8_t* qh = smem + a.u_off;                                    // [pair][I] permuted E4M3 (down)
+  double* yrow = reinterpret_cast<double*>(smem + a.u_off + a.yrow_off);  // [row tile][16][T] (down)
+  const int yrow_len = a.yrow_len;
   // this CTA's router rows (the same in every layer)
   const int row0 = E * cta / G;
-  const int nr = a.route ? E * (cta + 1) / G - row0 : 0;
-  // this CTA's gate/up tiles of the shared experts (the first tiles of every layer)
-  const int ns = cta < S * cpe ? (S * cpe - 1 - cta) / G + 1 : 0;
+  const int nrr = a.route ? E * (cta + 1) / G - row0 : 0;
+  // One token routed by this kernel always has k + S distinct experts, so
+  // the next layer's work split is known in advance and its first entries --
+  // gate/up tiles of the shared experts, the first tiles of every layer -- can
+  // be requested before its routing.
+  const bool predict = a.route && T == 1 && a.ep_lo == 0 && a.ep_hi == E;
+  Work pw{};
+  int npre = 0;  // entries of the coming layer already requested
+  if (predict) {
+    pw = plan_work(a, min(a.k, E) + S, cta, G, a.dpe);
+    npre = max(0, min(min(pw.g0 + pw.ng, S * cpe) - pw.g0, a.ns));
+  }
 
   MOE_TRACE_POINT(3, 0);
   // ---- before the dependency wait: the first layer's router rows and
-  // shared-expert tiles
+  // shared-expert tiles (weights only)
   LayerW lw = layer_ptrs(a, 0);
-  if (tid < NG) ug[tid] = 0;
-  if (tid < ND) ud[tid] = 0;
+  if (tid < kMaxNS) { iss[tid] = 0; arr[tid] = 0; }
   if (tid == 0) {
-    for (int s = 0; s < NG; ++s) mbar_init(&fg[s], 1);
-    for (int s = 0; s < ND; ++s) mbar_init(&fd[s], 1);
+    for (int s = 0; s < a.ns; ++s) mbar_init(&full[s], 1);
     mbar_init(&fr, 1);
     fence_mbar_init();
-    ur = 0;
+    s_riss = 0;
     s_abort = 0;
-    for (int s = 0; s < S; ++s) dist.expert[s] = E + s;  // rebuilt identically after routing
   }
-  for (int i = tid; i < kGroups * yg_len; i += kThreads) yg[i] = 0.0;
+  if (tid < MOE_MAX_SHARED) s_pre_expert[tid] = E + tid;
   __syncthreads();
-  if (tid == 0) {
-    if (nr > 0) copy_in(sm.rr, lw.Wr + static_cast<size_t>(row0) * H, nr * H * 2, &fr, &ur);
+  if (tid == 0 && nrr > 0) {
+    mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
+    bulk_g2s(rr, lw.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
+    s_riss = 1;
   }
-  if (warp < min(ns, NG) && lane == 0) issue_gu(a, sm, lw, dist.expert, warp, warp);
-  int npre = min(ns, NG);  // gate/up tiles of the coming layer already in flight
-  int gu_base = 0, dn_base = 0;
+  if (warp < npre && lane == 0) issue_entry(a, rg, lw, s_pre_expert, pw, warp, warp);
+  int ebase = 0;  // launch-wide number of this layer's entry 0
 
   pdl_wait();
   pdl_trigger();
   bool ok = true;
+  // tags of this launch's logits: launches so far (the previous launch's
+  // last CTA counted itself in before this one could start), layer
+  const unsigned tag0 = __ldcg(a.sync + kSyncEpoch) * 256u + 1u;
 
   for (int l = 0; l < L && ok; ++l) {
     MOE_TRACE_POINT(3, 1);
@@ -403,14 +619,14 @@ decode_kernel(DecodeArgs a) {
         if (stack) reinterpret_cast<uint4*>(rs)[u] = __ldcg(reinterpret_cast<const uint4*>(a.r_io) + u);
       }
       __syncthreads();
-    } else {
-      if (tid == 0 && !poll_geq_bounded(a.sync + kSyncY, static_cast<unsigned>(l * G), a.err)) {
+    } else if (kStack) {
+      // the previous layer's y: every CTA's rows, read as their tagged words arrive
+      if (!residual_norm(a, rs, a.ty + static_cast<size_t>((l - 1) & 1) * T * H / 2, tag0 + (l - 1), xb, red_d,
+                         den_s, &s_abort)) {
         ok = false;
         note_timeout(__LINE__, l, -1);
+        break;
       }
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      if (kStack) residual_norm(a, rs, a.ybuf + static_cast<size_t>((l - 1) & 1) * T * H, xb, red_d, den_s);
     }
     if (kDebug && a.dbg_x && cta == 0)
       for (int u = tid; u < T * H / 8; u += kThreads)
@@ -468,14 +684,13 @@ decode_kernel(DecodeArgs a) {
     float* w_l = a.w ? a.w + static_cast<size_t>(l) * T * a.k : nullptr;
     const LayerW lw_next = l + 1 < L ? layer_ptrs(a, l + 1) : lw;
     if (a.route) {
-      if (nr > 0 && !mbar_wait_bounded(&fr, l & 1, a.err)) {
+      if (nrr > 0 && !mbar_wait_bounded(&fr, l & 1, a.err)) {
         ok = false;
         if (tid == 0) note_timeout(__LINE__, l, -1);
       }
-      const uint16_t* rrows = reinterpret_cast<const uint16_t*>(sm.rr);
-      double* lpart = reinterpret_cast<double*>(smem + a.red_off + up128(static_cast<size_t>(T) * H * 2));
+      const uint16_t* rrows = reinterpret_cast<const uint16_t*>(rr);
       const int ql = H / 4;  // elements per quarter row
-      const int items = ok ? nr * T * 4 : 0;
+      const int items = ok ? nrr * T * 4 : 0;
       for (int it = warp; it < items; it += kWarps) {
         const int ri = it / (T * 4), tt = (it / 4) % T, qq = it % 4;
         const uint4* wrow = reinterpret_cast<const uint4*>(rrows + static_cast<size_t>(ri) * H + qq * ql);
@@ -486,30 +701,32 @@ decode_kernel(DecodeArgs a) {
         if (lane == 0) lpart[it] = acc;
       }
       __syncthreads();
-      for (int i = tid; i < nr * T && ok; i += kThreads) {
+      const unsigned tag = tag0 + static_cast<unsigned>(l);
+      for (int i = tid; i < nrr * T && ok; i += kThreads) {
         const int ri = i / T, tt = i % T;
         const double* p = lpart + (ri * T + tt) * 4;
         float lg = static_cast<float>((p[0] + p[1]) + (p[2] + p[3]));
         if (lw.bias) lg = __fadd_rn(lg, __ldg(lw.bias + row0 + ri));
-        __stcg(a.logits + static_cast<size_t>(tt) * E + row0 + ri, lg);
+        st_relaxed_u64(a.tlogits + static_cast<size_t>(tt) * E + row0 + ri,
+                       static_cast<unsigned long long>(tag) << 32 | __float_as_uint(lg));
       }
       __syncthreads();
       MOE_TRACE_POINT(3, 3);
-      if (tid == 0) {
-        __threadfence();
-        red_release_add_u32(a.sync + kSyncRoute, 1u);
-        // the router rows are used: the next layer's stream in meanwhile
-        if (l + 1 < L && nr > 0 && ok) copy_in(sm.rr, lw_next.Wr + static_cast<size_t>(row0) * H, nr * H * 2, &fr, &ur);
-        if (!poll_geq_bounded(a.sync + kSyncRoute, static_cast<unsigned>((l + 1) * G), a.err)) {
-          ok = false;
-          note_timeout(__LINE__, l, -1);
-        }
+      // the router rows are used: the next layer's stream in meanwhile
+      if (tid == 0 && l + 1 < L && nrr > 0 && ok) {
+        mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
+        bulk_g2s(rr, lw_next.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
+        ++s_riss;
+      }
+      if (warp < T && ok &&
+          !topk_warp(a.tlogits + static_cast<size_t>(warp) * E, tag, E, a.k, s_ids + warp * a.k, s_w + warp * a.k,
+                     a.err, &s_abort)) {
+        ok = false;
+        if (lane == 0) note_timeout(__LINE__, l, -1);
       }
       ok = __syncthreads_and(ok);
       if (!ok) break;
       MOE_TRACE_POINT(3, 4);
-      if (warp < T) topk_warp(a.logits + static_cast<size_t>(warp) * E, E, a.k, s_ids + warp * a.k, s_w + warp * a.k);
-      __syncthreads();
       if (cta == 0) {
         if (tid < T * a.k) {
           if (ids_l) ids_l[tid] = s_ids[tid];
@@ -527,20 +744,27 @@ decode_kernel(DecodeArgs a) {
       s_ids[lane] = __ldcg(a.ids + lane);
       s_w[lane] = __ldcg(a.w + lane);
     }
-    if (warp == 0) build_distinct(s_ids, s_w, T, a.k, E, S, dist, wsum, a.err, cta == 0 && !a.route);
+    if (warp == 0) build_distinct(s_ids, s_w, T, a.k, E, S, dist, wsum, a.err, cta == 0 && !a.route, a.ep_lo, a.ep_hi);
     __syncthreads();
     MOE_TRACE_POINT(3, 5);
 
-    // ---- this layer's work and its first copies (warp j issues entry j)
-    const int nd = dist.n;
-    const int ntiles = nd * cpe;
-    const int ng = cta < ntiles ? (ntiles - 1 - cta) / G + 1 : 0;
-    const int Stot = (H / 16) * nd;
-    const int q0 = slab_start(cta, Stot, G), q1 = slab_start(cta + 1, Stot, G);
-    const int nq = q1 - q0;
+    // ---- this layer's work and its first entries (warp w issues entries w, w + 16, ...)
+    const Work wk = plan_work(a, dist.n, cta, G, rg.dpe);
+    if (predict && wk.nd != pw.nd) {  // the requested entries would not be this layer's (never for routed T = 1)
+      if (tid == 0) atomicOr(a.err, kErrTimeout);
+      ok = false;
+      break;
+    }
+    // gate/up tiles first; the down slabs that also fit in the ring follow as
+    // soon as the CTA's first routed tile has landed (so they do not compete
+    // with the gate/up bytes, which the critical path waits for; the down
+    // bytes are needed only after the gate/up barrier)
+    const int first_routed = wk.ng > 0 && wk.g0 + wk.ng > S * cpe ? max(0, S * cpe - wk.g0) : -1;
+    const int dn_lo = max(wk.ng, npre), dn_hi = min(wk.cnt, rg.ns);
     if (lane == 0) {
-      for (int j = npre + warp; j < min(ng, NG); j += kWarps) issue_gu(a, sm, lw, dist.expert, j, gu_base + j);
-      for (int i = warp; i < min(nq, ND); i += kWarps) issue_dn(a, sm, lw, dist.expert, nd, q0 + i, dn_base + i);
+      for (int j = npre + warp; j < min(wk.ng, rg.ns); j += kWarps) issue_entry(a, rg, lw, dist.expert, wk, j, ebase + j);
+      if (first_routed < 0)
+        for (int j = dn_lo + warp; j < dn_hi; j += kWarps) issue_entry(a, rg, lw, dist.expert, wk, j, ebase + j);
     }
     // pair table of the down step (off the critical path): the (expert,
     // token) pairs in order, numbered by a ballot prefix count
@@ -548,7 +772,7 @@ decode_kernel(DecodeArgs a) {
       int base_p = 0;
       for (int i0 = 0; i0 < kMaxDistinct * kMaxTokGemv; i0 += 32) {
         const int i = i0 + lane, u = i / kMaxTokGemv, t = i % kMaxTokGemv;
-        const bool use = u < nd && t < T && (dist.mask[u] >> t & 1);
+        const bool use = u < wk.nd && t < T && (dist.mask[u] >> t & 1);
         const unsigned m = __ballot_sync(0xffffffffu, use);
         const int pi = base_p + __popc(m & ((1u << lane) - 1u));
         if (u < kMaxDistinct) pair_of[u][t] = use ? pi : -1;
@@ -562,87 +786,70 @@ decode_kernel(DecodeArgs a) {
     }
     MOE_TRACE_POINT(3, 6);
 
-    // ---- 3. gate/up + SwiGLU: group grp takes tiles grp, grp + 4, ...
+    // ---- 3. gate/up + SwiGLU: group grp takes tiles grp, grp + 4, ...; warp
+    // wq of the group the K quarter wq of each
     {
       const int g = lane >> 2, t4 = lane & 3;
-      const int nb = H / 32;
-      const int nbw = (nb + kGW - 1) / kGW;
-      const int b0 = wg * nbw, b1 = min(nb, b0 + nbw);
+      const int nbq = (nb + kQuarters - 1) / kQuarters;
+      const int b0 = min(nb, wq * nbq), b1 = min(nb, b0 + nbq);
       unsigned* amax_l = a.amax + static_cast<size_t>(l) * kMaxDistinct * kMaxTokGemv;
-      const int gbuf = kGW * 16 * T;  // doubles per partial buffer
-      for (int j = grp, n = 0; j < ng; j += kGroups, ++n) {
-        const int gidx = gu_base + j, s = gidx % NG;
-        const bool good = wait_slot(&fg[s], &ug[s], gidx / NG, a.err);
-        if (!good && lane == 0) note_timeout(__LINE__, l, gidx);
-        if (j < 8) MOE_TRACE_POINT(3, 20 + j);
-        const uint8_t* st = sm.gu + static_cast<size_t>(s) * gu_entry_bytes(H);
-        const int i = cta + G * j, u = i / cpe, f0 = (i % cpe) * kFeat;
-        const bool tok = g < T && (dist.mask[u] >> g & 1);
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        if (good) {
-          // kBatch blocks per step: their MMAs are all in flight before the
-          // first epilogue needs a result
-          for (int b = b0; b < b1; b += kBatch) {
-            float d[kBatch][4];
-            uint32_t sc[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-              const int bb = b + u < b1 ? b + u : b1 - 1;
-              const uint2 cw = *reinterpret_cast<const uint2*>(st + 256 * bb + 8 * lane);
-              sc[u] = *reinterpret_cast<const uint16_t*>(st + 256 * nb + 16 * bb + 2 * g);
-              const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
-              uint2 q = make_uint2(0u, 0u);
-              if (tok) q = *reinterpret_cast<const uint2*>(xq + static_cast<size_t>(g) * H + 32 * bb + 8 * t4);
-              mma_fp8(d[u], af, q.x, q.y);
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-              if (b + u >= b1) break;
-              const uint32_t ea = block_ebits(sc[u] & 0xFFu), eb = block_ebits(sc[u] >> 8);
-              acc[0] += scaled_block_f64(d[u][0], ea);
-              acc[2] += scaled_block_f64(d[u][2], eb);
-              if (T > 1) {
-                acc[1] += scaled_block_f64(d[u][1], ea);
-                acc[3] += scaled_block_f64(d[u][3], eb);
-              }
-            }
-          }
-        }
-        double* red = redd + static_cast<size_t>(grp * 2 + (n & 1)) * gbuf;
-        if (2 * t4 < T) {
-          red[(wg * 16 + g) * T + 2 * t4] = acc[0];
-          red[(wg * 16 + g + 8) * T + 2 * t4] = acc[2];
-          if (2 * t4 + 1 < T) {
-            red[(wg * 16 + g) * T + 2 * t4 + 1] = acc[1];
-            red[(wg * 16 + g + 8) * T + 2 * t4 + 1] = acc[3];
-          }
-        }
-        if (j < 8) MOE_TRACE_POINT(3, 28 + j);
-        if (group_sync_or(grp, !good || *reinterpret_cast<volatile int*>(&s_abort))) {
-          s_abort = 1;
+      const int pslot = kQuarters * 16 * T;  // partial sums per slot
+      for (int j = grp; j < wk.ng; j += kGroups) {
+        const int gidx = ebase + j, s = gidx % rg.ns;
+        if (!wait_entry(rg, gidx, a.err, &s_abort)) {
+          if (lane == 0) note_timeout(__LINE__, l, gidx);
           break;
         }
-        if (j < 8) MOE_TRACE_POINT(3, 48 + j);
-        if (wg == 1 && lane == 0 && j + NG < ng) issue_gu(a, sm, lw, dist.expert, j + NG, gidx + NG);
-        if (wg == 0) {
-          // lanes (feature f, token t) for f < 8, t < T
-          for (int o = lane; o < kFeat * T; o += 32) {
-            const int f = o / T, tt = o % T;
-            double gs = 0.0, us = 0.0;
-#pragma unroll
-            for (int w = 0; w < kGW; ++w) {
-              gs += red[(w * 16 + f) * T + tt];
-              us += red[(w * 16 + f + 8) * T + tt];
-            }
-            if (dist.mask[u] >> tt & 1) {
-              const double gv = static_cast<double>(xs[tt]) * gs;
-              const double uv = static_cast<double>(xs[tt]) * us;
-              const float hv = static_cast<float>(gv / (1.0 + exp(-gv)) * uv);
-              __stcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + f0 + f, hv);
-              const float m = fabsf(hv);
-              if (m > 0.f) atomicMax(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
-            }
+        if (j < 8 && wq == 0) MOE_TRACE_POINT(3, 20 + j);
+        if (j == first_routed && wq == 0 && lane == 0)
+          for (int jd = dn_lo; jd < dn_hi; ++jd) issue_entry(a, rg, lw, dist.expert, wk, jd, ebase + jd);
+        const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot;
+        const int i = wk.g0 + j, u = i / cpe, f0 = (i % cpe) * kFeat;
+        const bool tok = g < T && (dist.mask[u] >> g & 1);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_blocks<kTc>(st, nb, b0, b1, tok ? xq + static_cast<size_t>(g) * H + 8 * t4 : nullptr, acc);
+        float* red = redp + static_cast<size_t>(s) * pslot + wq * 16 * T;
+        if (2 * t4 < T) {
+          red[g * T + 2 * t4] = acc[0];
+          red[(g + 8) * T + 2 * t4] = acc[2];
+          if (!kT1 && 2 * t4 + 1 < T) {
+            red[g * T + 2 * t4 + 1] = acc[1];
+            red[(g + 8) * T + 2 * t4 + 1] = acc[3];
           }
+        }
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          __threadfence_block();
+          last = atomicAdd(&rg.arr[s], 1) == kQuarters - 1;
+          if (last) rg.arr[s] = 0;
+          __threadfence_block();
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __syncwarp();  // lane 0's acquire orders the other lanes' reads too
+        if (j < 8) MOE_TRACE_POINT(3, 28 + j);
+        // the 4 quarters' sums of feature f, token tt (lanes o = f * T + tt)
+        const float* rs4 = redp + static_cast<size_t>(s) * pslot;
+        double gs = 0.0, us = 0.0;
+        const int f = lane / T, tt = lane % T;
+        if (lane < kFeat * T) {
+#pragma unroll
+          for (int q = 0; q < kQuarters; ++q) {
+            gs += rs4[(q * 16 + f) * T + tt];
+            us += rs4[(q * 16 + f + 8) * T + tt];
+          }
+        }
+        __syncwarp();
+        // the slot is free: its next entry streams in while SwiGLU runs
+        if (lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
+        if (lane < kFeat * T && (dist.mask[u] >> tt & 1)) {
+          const double gv = static_cast<double>(xs[tt]) * gs;
+          const double uv = static_cast<double>(xs[tt]) * us;
+          const float hv = static_cast<float>(gv / (1.0 + exp(-gv)) * uv);
+          __stcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + f0 + f, hv);
+          const float m = fabsf(hv);
+          if (m > 0.f) atomicMax(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
         }
         if (j < 8) MOE_TRACE_POINT(3, 40 + j);
       }
@@ -650,13 +857,6 @@ decode_kernel(DecodeArgs a) {
     ok = __syncthreads_and(!s_abort);
     if (!ok) break;
     MOE_TRACE_POINT(3, 7);
-    gu_base += ng;
-    // every gate/up slot is free: the next layer's shared-expert tiles stream
-    // in during the down step
-    const LayerW lw_cur = lw;
-    lw = lw_next;
-    npre = l + 1 < L ? min(ns, NG) : 0;
-    if (warp < npre && lane == 0) issue_gu(a, sm, lw_next, dist.expert, warp, gu_base + warp);
     // every CTA's h and amax are needed by every CTA's down slabs
     if (tid == 0) {
       __threadfence();
@@ -670,15 +870,36 @@ decode_kernel(DecodeArgs a) {
     if (!ok) break;
     MOE_TRACE_POINT(3, 8);
 
-    // ---- 4. down + combine: group grp takes slabs grp, grp + 4, ...
-    uint16_t* y_l = (!stack && l == L - 1) ? a.y : a.ybuf + static_cast<size_t>(l & 1) * T * H;
+    // ---- 4. down + combine
+    // y of this layer: a plain layer's output (bf16), or a stacked layer's
+    // tagged words (two rows per word) that the next layer polls
+    uint16_t* y_l = a.y;
+    unsigned long long* ty_l = a.ty ? a.ty + static_cast<size_t>(l & 1) * T * H / 2 : nullptr;
+    const unsigned long long ytag = static_cast<unsigned long long>(tag0 + l) << 32;
+    const int nd = wk.nd, nq = wk.nq;
     if (nq > 0) {
       const int np = s_npairs;
       unsigned* amax_l = a.amax + static_cast<size_t>(l) * kMaxDistinct * kMaxTokGemv;
+      // every pair's h and amax in one round trip: the amax of pair tid and
+      // the first kHLoads float4 of h per thread are requested together
+      const int per = I / 4;
+      const int total4 = np * per;
+      float amx = 0.f;
+      if (tid < np) amx = __uint_as_float(__ldcg(amax_l + pair_d[tid] * kMaxTokGemv + pair_t[tid]));
+      float4 v[kHLoads];
+      int pr[kHLoads];
+#pragma unroll
+      for (int r = 0; r < kHLoads; ++r) {
+        const int idx = tid + r * kThreads;
+        pr[r] = idx < total4 ? idx / per : -1;
+        if (pr[r] >= 0)
+          v[r] = __ldcg(reinterpret_cast<const float4*>(
+                            a.h + (static_cast<size_t>(pair_d[pr[r]]) * kMaxTokGemv + pair_t[pr[r]]) * I) +
+                        (idx - pr[r] * per));
+      }
       if (tid < np) {
         const int u = pair_d[tid], tt = pair_t[tid];
-        const float amax = __uint_as_float(__ldcg(amax_l + u * kMaxTokGemv + tt));
-        const float shv = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+        const float shv = amx == 0.f ? 1.f : __fdiv_rn(amx, 448.f);
         shs[u][tt] = shv;
         coef[u][tt] = wsum[u][tt] * static_cast<double>(shv);
       }
@@ -686,26 +907,25 @@ decode_kernel(DecodeArgs a) {
         const int u = i / kMaxTokGemv, tt = i % kMaxTokGemv;
         if (pair_of[u][tt] < 0) coef[u][tt] = 0.0;
       }
-      // h of every pair -> registers (4 floats per load, 4 loads in flight),
-      // then FP8 codes in the fragment order (each group of 8 elements holds
-      // its even elements, then its odd ones)
-      const int per = I / 4;
-      const int total4 = np * per;
+      for (int i = tid; i < yrow_len; i += kThreads) yrow[i] = 0.0;
       __syncthreads();  // scales visible
-      for (int b4 = 0; b4 < total4; b4 += 4 * kThreads) {
-        float4 v[4];
-        int pr[4];
+      // FP8 codes of h in the fragment order (each group of 8 elements holds
+      // its even elements, then its odd ones); more than kHLoads float4 per
+      // thread (several tokens) take further rounds
+      for (int b4 = 0; b4 < total4; b4 += kHLoads * kThreads) {
+        if (b4 > 0) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int idx = b4 + tid + r * kThreads;
-          pr[r] = idx < total4 ? idx / per : -1;
-          if (pr[r] >= 0)
-            v[r] = __ldcg(reinterpret_cast<const float4*>(
-                              a.h + (static_cast<size_t>(pair_d[pr[r]]) * kMaxTokGemv + pair_t[pr[r]]) * I) +
-                          (idx - pr[r] * per));
+          for (int r = 0; r < kHLoads; ++r) {
+            const int idx = b4 + tid + r * kThreads;
+            pr[r] = idx < total4 ? idx / per : -1;
+            if (pr[r] >= 0)
+              v[r] = __ldcg(reinterpret_cast<const float4*>(
+                                a.h + (static_cast<size_t>(pair_d[pr[r]]) * kMaxTokGemv + pair_t[pr[r]]) * I) +
+                            (idx - pr[r] * per));
+          }
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < kHLoads; ++r) {
           if (pr[r] < 0) continue;
           const int j = 4 * (b4 + tid + r * kThreads - pr[r] * per);
           const float shv = shs[pair_d[pr[r]]][pair_t[pr[r]]];
@@ -713,16 +933,16 @@ decode_kernel(DecodeArgs a) {
           const uint32_t c2 = f32_to_e4m3(__fdiv_rn(v[r].z, shv)), c3 = f32_to_e4m3(__fdiv_rn(v[r].w, shv));
           // elements j..j+3 (j % 4 == 0): the two even ones go to bytes
           // o, o+1 of the group's even half, the two odd ones to the odd half
-          uint8_t* grp = qh + static_cast<size_t>(pr[r]) * I + (j & ~7);
+          uint8_t* gp = qh + static_cast<size_t>(pr[r]) * I + (j & ~7);
           const int o = (j & 4) >> 1;
-          *reinterpret_cast<uint16_t*>(grp + o) = static_cast<uint16_t>(c0 | c2 << 8);
-          *reinterpret_cast<uint16_t*>(grp + 4 + o) = static_cast<uint16_t>(c1 | c3 << 8);
+          *reinterpret_cast<uint16_t*>(gp + o) = static_cast<uint16_t>(c0 | c2 << 8);
+          *reinterpret_cast<uint16_t*>(gp + 4 + o) = static_cast<uint16_t>(c1 | c3 << 8);
         }
       }
       __syncthreads();
       MOE_TRACE_POINT(3, 9);
-      // debug copies by the CTA holding slab 0 (every CTA with down work has all of qh)
-      if (kDebug && q0 == 0 && (a.dbg.qh || a.dbg.h || a.dbg.sh)) {
+      // debug copies by the CTA holding row tile 0 (every CTA with down work has all of qh)
+      if (kDebug && wk.r0 == 0 && (a.dbg.qh || a.dbg.h || a.dbg.sh)) {
         const int Sl = a.k + S;
         for (int pp = warp; pp < T * Sl; pp += kWarps) {
           const int tt = pp / Sl, si = pp % Sl;
@@ -742,150 +962,104 @@ decode_kernel(DecodeArgs a) {
         }
       }
 
+      // slab items: item it = (slab it / dsplit, K part it % dsplit), warp it mod 16
       const int g = lane >> 2, t4 = lane & 3;
-      const int nbI = I / 32;
-      const int bpw = (nbI + kGW - 1) / kGW;
-      const int b0 = wg * bpw, b1 = min(nbI, b0 + bpw);
-      const int rt0 = q0 / nd;
-      const int gbuf = kGW * 16 * T;
-      double* ygl = yg + static_cast<size_t>(grp) * yg_len;
-      for (int i = grp, n = 0; i < nq; i += kGroups, ++n) {
-        const int didx = dn_base + i, s = didx % ND;
-        const bool good = wait_slot(&fd[s], &ud[s], didx / ND, a.err);
-        if (!good && lane == 0) note_timeout(__LINE__, l, didx);
-        if (i < 8) MOE_TRACE_POINT(3, 12 + (i >> 2));
-        const int q = q0 + i, u = q % nd, lr = q / nd - rt0;
-        const uint8_t* st = sm.dn + static_cast<size_t>(s) * dn_entry_bytes(I);
-        const int pg = g < T ? pair_of[u][g] : -1;
-        const double c0 = coef[u][(2 * t4) & 3], c1 = coef[u][(2 * t4 + 1) & 3];
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        if (good) {
-          for (int b = b0; b < b1; b += kBatch) {
-            float d[kBatch][4];
-            uint32_t sc[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-              const int bb = b + u < b1 ? b + u : b1 - 1;
-              const uint2 cw = *reinterpret_cast<const uint2*>(st + 256 * bb + 8 * lane);
-              sc[u] = *reinterpret_cast<const uint16_t*>(st + 256 * nbI + 16 * bb + 2 * g);
-              const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
-              uint2 qv = make_uint2(0u, 0u);
-              if (pg >= 0) qv = *reinterpret_cast<const uint2*>(qh + static_cast<size_t>(pg) * I + 32 * bb + 8 * t4);
-              mma_fp8(d[u], af, qv.x, qv.y);
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-              if (b + u >= b1) break;
-              const uint32_t ea = block_ebits(sc[u] & 0xFFu), eb = block_ebits(sc[u] >> 8);
-              acc[0] = fma(scaled_block_f64(d[u][0], ea), c0, acc[0]);
-              acc[2] = fma(scaled_block_f64(d[u][2], eb), c0, acc[2]);
-              if (T > 1) {
-                acc[1] = fma(scaled_block_f64(d[u][1], ea), c1, acc[1]);
-                acc[3] = fma(scaled_block_f64(d[u][3], eb), c1, acc[3]);
-              }
-            }
-          }
-        }
-        double* red = redd + static_cast<size_t>(grp * 2 + (n & 1)) * gbuf;
-        if (2 * t4 < T) {
-          red[(wg * 16 + g) * T + 2 * t4] = acc[0];
-          red[(wg * 16 + g + 8) * T + 2 * t4] = acc[2];
-          if (2 * t4 + 1 < T) {
-            red[(wg * 16 + g) * T + 2 * t4 + 1] = acc[1];
-            red[(wg * 16 + g + 8) * T + 2 * t4 + 1] = acc[3];
-          }
-        }
-        if (group_sync_or(grp, !good || *reinterpret_cast<volatile int*>(&s_abort))) {
-          s_abort = 1;
+      const int ds = wk.dsplit;
+      const int bpp = (nbI + ds - 1) / ds;
+      for (int it = warp; it < nq * ds; it += kWarps) {
+        const int k = it / ds, part = it % ds;
+        const int j = wk.ng + k / rg.dpe, gidx = ebase + j, s = gidx % rg.ns;
+        if (!wait_entry(rg, gidx, a.err, &s_abort)) {
+          if (lane == 0) note_timeout(__LINE__, l, gidx);
           break;
         }
-        if (wg == 1 && lane == 0 && i + ND < nq) issue_dn(a, sm, lw_cur, dist.expert, nd, q + ND, didx + ND);
-        if (wg == 0)
-          for (int o = lane; o < 16 * T; o += 32) {
-            const int row = o / T, tt = o % T;
-            double sum = 0.0;
-#pragma unroll
-            for (int w = 0; w < kGW; ++w) sum += red[(w * 16 + row) * T + tt];
-            ygl[(lr * 16 + row) * T + tt] += sum;
+        if (it < 16) MOE_TRACE_POINT(3, 12 + (it >> 2));
+        const int u = k % nd, lr = k / nd;
+        const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot + (k % rg.dpe) * dn_entry_bytes(I);
+        const int pg = g < T ? pair_of[u][g] : -1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int b0 = min(nbI, part * bpp), b1 = min(nbI, b0 + bpp);
+        tile_blocks<kTc>(st, nbI, b0, b1, pg >= 0 ? qh + static_cast<size_t>(pg) * I + 8 * t4 : nullptr, acc);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          last = atomicAdd(&rg.arr[s], 1) == entry_items(rg, wk, j) - 1;
+          if (last) rg.arr[s] = 0;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last && lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
+        // rows g, g + 8 of tokens 2 t4, 2 t4 + 1, times w * s_h, into the
+        // float64 row sums (every expert of the row tile adds here)
+        double* yr = yrow + static_cast<size_t>(lr) * 16 * T;
+        if (2 * t4 < T) {
+          const double c0 = coef[u][2 * t4];
+          if (c0 != 0.0) {
+            atomicAdd(yr + g * T + 2 * t4, static_cast<double>(acc[0]) * c0);
+            atomicAdd(yr + (g + 8) * T + 2 * t4, static_cast<double>(acc[2]) * c0);
           }
+          if (!kT1 && 2 * t4 + 1 < T) {
+            const double c1 = coef[u][2 * t4 + 1];
+            if (c1 != 0.0) {
+              atomicAdd(yr + g * T + 2 * t4 + 1, static_cast<double>(acc[1]) * c1);
+              atomicAdd(yr + (g + 8) * T + 2 * t4 + 1, static_cast<double>(acc[3]) * c1);
+            }
+          }
+        }
       }
       ok = __syncthreads_and(!s_abort);
       MOE_TRACE_POINT(3, 10);
-      // finish the CTA's row tiles: owned ones directly; the first and last,
-      // when shared with a neighbouring CTA, through the float64 accumulators
-      // (whichever CTA adds last rounds them)
-      const int nrt = ok ? (q1 - 1) / nd - rt0 + 1 : 0;
-      const int row = tid / T, tt = tid % T;
-      int shared_lr[2] = {-1, -1};
-      int nsh = 0;
-      for (int lr = 0; lr < nrt; ++lr) {
-        const int r = rt0 + lr;
-        const int qa = r * nd, qb = qa + nd;
-        const bool owned = qa >= q0 && qb <= q1;
-        if (tid < 16 * T) {
-          const size_t yi = static_cast<size_t>(tt) * H + 16 * r + row;
-          double acc = 0.0;
-          for (int gg = 0; gg < kGroups; ++gg) {
-            double& v = yg[static_cast<size_t>(gg) * yg_len + (lr * 16 + row) * T + tt];
-            acc += v;
-            v = 0.0;
-          }
-          if (owned) y_l[yi] = f64_to_bf16_rne(acc);
-          else atomicAdd(a.yacc + yi, acc);
+      // the CTA's rows of y, each complete: a stacked layer publishes them as
+      // tagged words (two rows of one token per word), a plain layer as bf16
+      if (ok && stack) {
+        for (int i = tid; i < wk.nr * 8 * T; i += kThreads) {
+          const int lr = i / (8 * T), rp = (i / T) % 8, tt = i % T;
+          const double y0 = yrow[(lr * 16 + 2 * rp) * T + tt], y1 = yrow[(lr * 16 + 2 * rp + 1) * T + tt];
+          st_relaxed_u64(ty_l + (static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + 2 * rp) / 2,
+                         ytag | f64_to_bf16_rne(y0) | static_cast<unsigned long long>(f64_to_bf16_rne(y1)) << 16);
         }
-        if (!owned) {
-          if (nsh == 0) shared_lr[0] = lr;
-          else shared_lr[1] = lr;
-          ++nsh;
+      } else if (ok && a.y32) {  // the part of y this call's experts contribute, not yet rounded
+        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
+          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
+          a.y32[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = static_cast<float>(yrow[(lr * 16 + row) * T + tt]);
         }
-      }
-      if (nsh > 0) {
-        __syncthreads();
-        if (tid == 0) {
-          __threadfence();
-          unsigned old[2] = {0u, 0u};
-          int nc[2] = {0, 0};
-          for (int i = 0; i < nsh && i < 2; ++i) {
-            const int r = rt0 + shared_lr[i];
-            const int c1 = slab_owner(r * nd, Stot, G), c2 = slab_owner(r * nd + nd - 1, Stot, G);
-            for (int c = c1; c <= c2; ++c) nc[i] += slab_start(c + 1, Stot, G) > slab_start(c, Stot, G);
-            old[i] = atomicAdd(a.tile_cnt + r, 1u);
-          }
-          s_last[0] = nsh > 0 && old[0] == static_cast<unsigned>(nc[0] - 1);
-          s_last[1] = nsh > 1 && old[1] == static_cast<unsigned>(nc[1] - 1);
-          if (s_last[0] || s_last[1]) __threadfence();
-        }
-        __syncthreads();
-        for (int i = 0; i < nsh && i < 2; ++i) {
-          if (!s_last[i]) continue;
-          const int r = rt0 + shared_lr[i];
-          if (tid < 16 * T) {
-            const size_t yi = static_cast<size_t>(tt) * H + 16 * r + row;
-            y_l[yi] = f64_to_bf16_rne(__ldcg(a.yacc + yi));
-            a.yacc[yi] = 0.0;
-          }
-          if (tid == 0) a.tile_cnt[r] = 0u;
+      } else if (ok) {
+        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
+          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
+          y_l[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = f64_to_bf16_rne(yrow[(lr * 16 + row) * T + tt]);
         }
       }
     }
-    dn_base += nq;
+    if (nq == 0 && wk.nr > 0 && ok) {
+      // no expert of this call contributes (every id skipped and no shared
+      // expert): the CTA's rows of y are zero
+      if (stack) {
+        for (int i = tid; i < wk.nr * 8 * T; i += kThreads) {
+          const int lr = i / (8 * T), rp = (i / T) % 8, tt = i % T;
+          st_relaxed_u64(ty_l + (static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + 2 * rp) / 2, ytag);
+        }
+      } else {
+        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
+          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
+          const size_t yi = static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row;
+          if (a.y32) a.y32[yi] = 0.f;
+          else y_l[yi] = 0;
+        }
+      }
+    }
+    ebase += wk.cnt;
     MOE_TRACE_POINT(3, 11);
-    // ---- 5. y of this layer complete (for the next layer or the final norm)
+    // ---- every slot is free: the next layer's first entries (shared-expert
+    // tiles) stream in
     __syncthreads();
-    if ((stack || l + 1 < L) && tid == 0) {
-      __threadfence();
-      red_release_add_u32(a.sync + kSyncY, 1u);
-    }
+    lw = lw_next;
+    if (l + 1 < L && ok && predict && warp < npre && lane == 0)
+      issue_entry(a, rg, lw_next, s_pre_expert, pw, warp, ebase + warp);
   }
 
   // ---- the stack's final residual and normalised x (CTA 0)
   if (kStack && ok && cta == 0) {
-    if (tid == 0 && !poll_geq_bounded(a.sync + kSyncY, static_cast<unsigned>(L * G), a.err)) {
-      ok = false;
-      note_timeout(__LINE__, L, -1);
-    }
-    if (__syncthreads_and(ok)) {
-      residual_norm(a, rs, a.ybuf + static_cast<size_t>((L - 1) & 1) * T * H, xb, red_d, den_s);
+    if (residual_norm(a, rs, a.ty + static_cast<size_t>((L - 1) & 1) * T * H / 2, tag0 + (L - 1), xb, red_d, den_s,
+                      &s_abort)) {
       for (int u = tid; u < T * H / 8; u += kThreads) {
         reinterpret_cast<uint4*>(a.r_io)[u] = reinterpret_cast<const uint4*>(rs)[u];
         reinterpret_cast<uint4*>(a.x_io)[u] = reinterpret_cast<const uint4*>(xb)[u];
@@ -897,9 +1071,8 @@ decode_kernel(DecodeArgs a) {
   // wait some may not have been consumed; the last use of every slot is
   // waited for, which returns at once when it completed)
   __syncthreads();
-  if (tid < NG && ug[tid] > 0) mbar_wait_bounded(&fg[tid], (ug[tid] - 1) & 1, nullptr);
-  if (tid >= 32 && tid < 32 + ND && ud[tid - 32] > 0) mbar_wait_bounded(&fd[tid - 32], (ud[tid - 32] - 1) & 1, nullptr);
-  if (tid == 64 && ur > 0) mbar_wait_bounded(&fr, (ur - 1) & 1, nullptr);
+  if (tid < a.ns && iss[tid] > 0) mbar_wait_bounded(&full[tid], (iss[tid] - 1) & 1, nullptr);
+  if (tid == 64 && s_riss > 0) mbar_wait_bounded(&fr, (s_riss - 1) & 1, nullptr);
   // ---- the last CTA clears the per-call counters
   __syncthreads();
   if (tid == 0) {
@@ -912,10 +1085,9 @@ decode_kernel(DecodeArgs a) {
     __threadfence();
     for (int i = tid; i < L * kMaxDistinct * kMaxTokGemv; i += kThreads) a.amax[i] = 0u;
     if (tid == 0) {
-      a.sync[kSyncRoute] = 0u;
       a.sync[kSyncGU] = 0u;
-      a.sync[kSyncY] = 0u;
       a.sync[kSyncExit] = 0u;
+      a.sync[kSyncEpoch] += 1u;  // the next launch's tags differ from every tag of this one
     }
   }
 }
@@ -944,83 +1116,110 @@ cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaS
 }
 
 // Shared-memory plan of one call; returns false when the shapes do not fit.
+// Dynamic shared memory, in order: the ring [ns][slot]; the router rows; the
+// FP8 x; the residual (stacks); then one region used in turn by the layer
+// start (bf16 x + router partial sums), gate/up (partial sums per slot) and
+// down (FP8 h of every pair + float64 row accumulators).
 bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   const int H = a.H, I = a.I, T = a.T;
   if (T < 1 || T > kMaxTokGemv || n_ctas < 1 || a.L < 1) return false;
   const int R = H / 16;
-  const size_t xq = up128(static_cast<size_t>(T) * H);
+  const size_t gb = gu_entry_bytes(H), db = dn_entry_bytes(I);
+  const size_t slot = up128(gb > db ? gb : db);
+  a.slot_bytes = static_cast<int>(slot);
+  a.dpe = static_cast<int>(slot / db);
   const int rr_max = a.route ? (a.E + n_ctas - 1) / n_ctas : 0;
   const size_t rr = up128(static_cast<size_t>(rr_max) * H * 2);
-  size_t red = static_cast<size_t>(kGroups) * 2 * kGW * 16 * T * 8;  // group partials, double-buffered
-  const size_t x_need = up128(static_cast<size_t>(T) * H * 2) + static_cast<size_t>(rr_max) * T * 4 * 8;
-  if (x_need > red) red = x_need;
-  red = up128(red);
-  const size_t qh = up128(static_cast<size_t>(T) * (a.k + a.n_shared) * I);
-  const int nrt = (R + n_ctas - 1) / n_ctas + 2;
-  a.yrow_len = nrt * 16 * T;
-  const size_t yrow = up128(static_cast<size_t>(kGroups) * a.yrow_len * 8);
+  const size_t xq = up128(static_cast<size_t>(T) * H);
   const size_t rs = a.r_io ? up128(static_cast<size_t>(T) * H * 2) : 0;
-  const size_t other = rr + xq + red + qh + yrow + rs;
-  if (static_cast<size_t>(smem_budget) <= other) return false;
-  const size_t rings = static_cast<size_t>(smem_budget) - other;
-  const size_t gb = gu_entry_bytes(H), db = dn_entry_bytes(I);
-  // the most the CTA can use: its gate/up tiles and down slabs of one call
-  const int max_d = T * a.k + a.n_shared;
-  const int gu_max = (max_d * (I / kFeat) + n_ctas - 1) / n_ctas;
-  const int dn_max = (max_d * R + n_ctas - 1) / n_ctas;
-  // down slots first (they stay resident while gate/up runs), gate/up takes the rest
-  int nd_slots = dn_max < kMaxND ? dn_max : kMaxND;
-  while (nd_slots > 4 && nd_slots * db + 4 * gb > rings) --nd_slots;
-  if (nd_slots < 1) nd_slots = 1;
-  if (nd_slots * db + gb > rings) return false;
-  int ng_slots = static_cast<int>((rings - nd_slots * db) / gb);
-  if (ng_slots > gu_max) ng_slots = gu_max;
-  if (ng_slots > kMaxNG) ng_slots = kMaxNG;
-  if (ng_slots < 1) ng_slots = 1;
-  a.ng_slots = ng_slots;
-  a.nd_slots = nd_slots;
-  size_t off = 0;
-  a.dn_off = static_cast<int>(off += static_cast<size_t>(ng_slots) * gb);
-  a.rr_off = static_cast<int>(off += static_cast<size_t>(nd_slots) * db);
-  off = up128(off);
-  a.rr_off = static_cast<int>(off);
-  a.xq_off = static_cast<int>(off += rr);
-  a.red_off = static_cast<int>(off += xq);
-  a.qh_off = static_cast<int>(off += red);
-  a.yrow_off = static_cast<int>(off += qh);
-  a.rs_off = static_cast<int>(off += yrow);
-  off += rs;
-  a.smem_bytes = static_cast<int>(off);
-  return a.smem_bytes <= smem_budget;
+  // layer start: bf16 x, router partial sums
+  a.lpart_off = static_cast<int>(up128(static_cast<size_t>(T) * H * 2));
+  const size_t u_start = a.lpart_off + up128(static_cast<size_t>(rr_max) * T * 4 * 8);
+  // down: FP8 h of every pair, the float64 sums of the CTA's row tiles
+  const int nrt = R / n_ctas + 1;
+  a.yrow_len = nrt * 16 * T;
+  a.yrow_off = static_cast<int>(up128(static_cast<size_t>(T) * (a.k + a.n_shared) * I));
+  const size_t u_down = a.yrow_off + up128(static_cast<size_t>(a.yrow_len) * 8);
+  // the most entries one CTA can have in a layer (slots beyond it are unused)
+  const size_t max_d = static_cast<size_t>(T) * a.k + a.n_shared;
+  const size_t bytes = max_d * (I / kFeat) * gb + static_cast<size_t>(R) * max_d * db;
+  const int ent_max = static_cast<int>((bytes / n_ctas + gb - 1) / gb + 2 + (nrt * max_d + a.dpe - 1) / a.dpe);
+  for (int ns = kMaxNS; ns >= 2; --ns) {
+    if (ns > ent_max && ns > 2) continue;
+    const size_t u_gu = up128(static_cast<size_t>(ns) * kQuarters * 16 * T * 4);
+    size_t u = u_start > u_down ? u_start : u_down;
+    if (u_gu > u) u = u_gu;
+    size_t off = static_cast<size_t>(ns) * slot;
+    a.rr_off = static_cast<int>(off);
+    off += rr;
+    a.xq_off = static_cast<int>(off);
+    off += xq;
+    a.rs_off = static_cast<int>(off);
+    off += rs;
+    a.u_off = static_cast<int>(off);
+    off += u;
+    if (off <= static_cast<size_t>(smem_budget)) {
+      a.ns = ns;
+      a.smem_bytes = static_cast<int>(off);
+      return true;
+    }
+  }
+  return false;
 }
+
+namespace {
+
+const void* const kDecodeFns[8] = {
+    reinterpret_cast<const void*>(decode_kernel<false, false, false>),
+    reinterpret_cast<const void*>(decode_kernel<false, false, true>),
+    reinterpret_cast<const void*>(decode_kernel<false, true, false>),
+    reinterpret_cast<const void*>(decode_kernel<false, true, true>),
+    reinterpret_cast<const void*>(decode_kernel<true, false, false>),
+    reinterpret_cast<const void*>(decode_kernel<true, false, true>),
+    reinterpret_cast<const void*>(decode_kernel<true, true, false>),
+    reinterpret_cast<const void*>(decode_kernel<true, true, true>)};
+
+}  // namespace
 
 const void* decode_fn(const DecodeArgs& a) {
   const bool dbg = a.dbg.xq || a.dbg.xs || a.dbg.h || a.dbg.qh || a.dbg.sh || a.dbg_x;
-  if (a.r_io) return dbg ? reinterpret_cast<const void*>(decode_kernel<true, true>)
-                         : reinterpret_cast<const void*>(decode_kernel<true, false>);
-  return dbg ? reinterpret_cast<const void*>(decode_kernel<false, true>)
-             : reinterpret_cast<const void*>(decode_kernel<false, false>);
+  return kDecodeFns[(a.r_io ? 4 : 0) + (dbg ? 2 : 0) + (a.T == 1 ? 1 : 0)];
 }
 
 cudaError_t launch_decode(const DecodeArgs& a_in, int n_ctas, cudaStream_t stream) {
-  // largest dynamic shared-memory size set so far, per device
+  // per device: the largest dynamic shared-memory size set so far, and the
+  // largest size whose co-residency (one CTA of every kernel variant per SM,
+  // grid <= SMs) has been checked
   static std::atomic<int> configured[kMaxDevices];
+  static std::atomic<int> resident_ok[kMaxDevices];
   DecodeArgs a = a_in;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (a.smem_bytes > configured[dev].load()) {
-    const void* fns[4] = {reinterpret_cast<const void*>(decode_kernel<false, false>),
-                          reinterpret_cast<const void*>(decode_kernel<false, true>),
-                          reinterpret_cast<const void*>(decode_kernel<true, false>),
-                          reinterpret_cast<const void*>(decode_kernel<true, true>)};
-    for (const void* f : fns) {
+    for (const void* f : kDecodeFns) {
       err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
       if (err != cudaSuccess) return err;
     }
     int cur = configured[dev].load();
     while (cur < a.smem_bytes && !configured[dev].compare_exchange_weak(cur, a.smem_bytes)) {
+    }
+  }
+  if (a.smem_bytes > resident_ok[dev].load()) {
+    // the grid-wide waits need every CTA resident at once
+    int sms = 0;
+    err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    if (n_ctas > sms) return cudaErrorCooperativeLaunchTooLarge;
+    for (const void* f : kDecodeFns) {
+      int per_sm = 0;
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kThreads, static_cast<size_t>(a.smem_bytes));
+      if (err != cudaSuccess) return err;
+      if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    }
+    int cur = resident_ok[dev].load();
+    while (cur < a.smem_bytes && !resident_ok[dev].compare_exchange_weak(cur, a.smem_bytes)) {
     }
   }
   void* kargs[] = {&a};
@@ -1029,11 +1228,7 @@ cudaError_t launch_decode(const DecodeArgs& a_in, int n_ctas, cudaStream_t strea
 
 int decode_static_smem() {
   int most = 0;
-  const void* fns[4] = {reinterpret_cast<const void*>(decode_kernel<false, false>),
-                        reinterpret_cast<const void*>(decode_kernel<false, true>),
-                        reinterpret_cast<const void*>(decode_kernel<true, false>),
-                        reinterpret_cast<const void*>(decode_kernel<true, true>)};
-  for (const void* f : fns) {
+  for (const void* f : kDecodeFns) {
     cudaFuncAttributes attr{};
     if (cudaFuncGetAttributes(&attr, f) != cudaSuccess) return -1;
     if (static_cast<int>(attr.sharedSizeBytes) > most) most = static_cast<int>(attr.sharedSizeBytes);

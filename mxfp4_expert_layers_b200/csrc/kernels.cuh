@@ -26,24 +26,29 @@ struct RouteArgs {
   int32_t* ids;
   float* w;
   int32_t* counts;
+  const float* wnorm;   // [E + 1] router row norms and their maximum (many-token router)
+  int* err;             // device-side error bits
   // L2 prefetch of the shared experts for the expert kernels that follow
   int prefetch_shared;
   const uint8_t* w13;   // packed
   const uint8_t* w2;    // packed
 };
-// T > kRouteGemmMinTokens: logits GEMM on the FP64 tensor-core path + a
-// top-k kernel; otherwise one fused launch (programmatic dependent launch).
+// T > kRouteGemmMinTokens: approximate logits on the BF16 tensor cores, then
+// an exact recomputation of every expert near each token's top-k threshold
+// (filter, then verify); otherwise one fused launch (programmatic dependent
+// launch).
 constexpr int kRouteGemmMinTokens = 32;
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 int route_tiles(int T);
+// Router row norms for the many-token router: wnorm [E + 1] (the maximum last).
+cudaError_t launch_route_norms(const uint16_t* Wr, int E, int H, float* wnorm, cudaStream_t stream);
 
 // Fused decode pass, T <= MOE_GEMV_MAX_TOKENS (decode.cu): one persistent
 // launch for one layer or a chained stack of layers (routing optional for a
 // single layer; required for a stack).
-constexpr int kSyncRoute = 0;   // grid arrive/wait counter of the routing step
 constexpr int kSyncExit = 1;    // CTAs finished
 constexpr int kSyncGU = 2;      // CTAs whose gate/up tiles are finished
-constexpr int kSyncY = 3;       // CTAs whose part of y is written
+constexpr int kSyncEpoch = 4;   // launches completed (tags of the logits exchange)
 constexpr int kSyncWords = 64;
 constexpr int kMaxStackLayers = 128;
 struct LayerW {                 // one layer's weights (device pointers)
@@ -56,6 +61,7 @@ struct DecodeArgs {
   int H, I, E, k, n_shared, T;
   int L;                // layers (1 for moe_decode / moe_forward)
   int route;            // 1: routing computed inside (ids, w, counts are outputs)
+  int ep_lo, ep_hi;     // routed experts this call runs (0, E unless the layer is split over GPUs)
   LayerW layer0;        // the layer when `layers` is null
   const LayerW* layers; // [L] device array (stacks)
   const uint16_t* x;    // [T][H] input of the first layer
@@ -66,20 +72,22 @@ struct DecodeArgs {
   float* w;             // [L][T][k]
   int32_t* counts;      // [E] or null (single routed layer)
   uint16_t* y;          // [T][H] output of a plain layer
+  float* y32;           // [T][H] float32 part of y from this call's experts (replaces y), or null
   // workspace; the counters and accumulators are zero between calls
-  float* logits;        // [T][E]
+  unsigned long long* tlogits;  // [kMaxTokGemv][E] logit bits | tag << 32 (zero before the first call)
   float* h;             // [kMaxDistinct][kMaxTokGemv][I]
   unsigned* amax;       // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;       // [kSyncWords]
-  unsigned* tile_cnt;   // [H/16]
-  double* yacc;         // [kMaxTokGemv][H]
-  uint16_t* ybuf;       // [2][T][H] y of stacked layers
+  unsigned long long* ty;  // [2][T][H/2] y of stacked layers: two bf16 | tag << 32 (zero before the first call)
   int* err;
   moe_debug dbg;        // plain layer only
   uint16_t* dbg_x;      // [L][T][H] input x of every layer, or null
-  // shared-memory plan (decode_plan)
-  int ng_slots, nd_slots;  // gate/up and down ring slots
-  int dn_off, rr_off, xq_off, red_off, qh_off, yrow_off, rs_off, yrow_len, smem_bytes;
+  // shared-memory plan (decode_plan): the weight ring (ns slots of
+  // slot_bytes, a down entry holds dpe slabs), then the regions at the
+  // given byte offsets; u_off starts the region shared by the layer start,
+  // gate/up and down (lpart_off, yrow_off relative to it)
+  int ns, slot_bytes, dpe;
+  int rr_off, xq_off, rs_off, u_off, lpart_off, yrow_off, yrow_len, smem_bytes;
 };
 bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget);
 cudaError_t launch_decode(const DecodeArgs& a, int n_ctas, cudaStream_t stream);
@@ -184,6 +192,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, int n_sms, cudaStream_t stream,
 // Per-row FP8 quantisation (quant.cu)
 cudaError_t launch_quantize_rows(const float* v, int rows, int cols, uint8_t* q, float* s,
                                  cudaStream_t stream);
+// float32 -> BF16 bits, round to nearest even (quant.cu)
+cudaError_t launch_round_bf16(const float* v, size_t n, uint16_t* out, cudaStream_t stream);
 
 // Harness step for chained layers (norm.cu)
 cudaError_t launch_residual_rmsnorm(uint16_t* r, const uint16_t* y, uint16_t* x_next, int T,

@@ -13,6 +13,9 @@ struct moe_handle_s {
   int max_tokens;
   int last_path;
   int prefill_kernel;  // MOE_PREFILL_*
+  bool ep;             // a part of a layer split over GPUs (moe_create_ep)
+  int ep_lo, ep_hi;    // its routed experts
+  bool ep_shared;      // it adds the shared experts
   bool tc_ok;          // the tcgen05 grouped GEMMs can run (shape, tensor maps)
   void* ws;
   size_t ws_bytes;
@@ -24,8 +27,8 @@ struct moe_handle_s {
   unsigned* amax;      // [kMaxDistinct][kMaxTokGemv]
   float* h;            // [kMaxDistinct][kMaxTokGemv][I]
   unsigned* sync;      // [kSyncWords]
-  unsigned* tile_cnt;  // [H/16]
-  double* yacc;        // [kMaxTokGemv][H]
+  unsigned long long* tlogits;  // [kMaxTokGemv][E] tagged logits of the fused decode kernel
+  float* wnorm;        // [E + 1] router row norms (many-token router), or null
   int n_sms;
   int smem_budget;     // dynamic shared memory available to the decode kernel
   moe::PrefillArgs pf; // workspace views of the many-token path (max_tokens > 4)
@@ -93,8 +96,8 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const size_t n_amax = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * I * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
-  const size_t n_tcnt = up256(static_cast<size_t>(cfg->hidden / 16) * 4);
-  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * cfg->hidden * 8);
+  const size_t n_tlog = up256(static_cast<size_t>(moe::kMaxTokGemv) * E * 8);
+  const size_t n_wnorm = max_tokens > moe::kRouteGemmMinTokens ? up256(static_cast<size_t>(E + 1) * 4) : 0;
   // the many-token path: pairs P = max_tokens * (k + S)
   const size_t T = static_cast<size_t>(max_tokens), H = cfg->hidden, NE = E + cfg->n_shared;
   const size_t P = T * (cfg->top_k + cfg->n_shared);
@@ -120,7 +123,7 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   size_t n_pf = 0;
   if (many)
     for (size_t v : pf_sizes) n_pf += v;
-  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tcnt + n_yacc + n_pf;
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tlog + n_wnorm + n_pf;
   int dev = 0, optin = 0;
   const int static_smem = moe::decode_static_smem();
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -149,8 +152,8 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
   h->h = reinterpret_cast<float*>(p); p += n_h;
   h->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
-  h->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
-  h->yacc = reinterpret_cast<double*>(p); p += n_yacc;
+  h->tlogits = reinterpret_cast<unsigned long long*>(p); p += n_tlog;
+  h->wnorm = n_wnorm ? reinterpret_cast<float*>(p) : nullptr; p += n_wnorm;
   h->pf = moe::PrefillArgs{};
   if (many) {
     moe::PrefillArgs& f = h->pf;
@@ -183,6 +186,12 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     f.w13 = weights->w13; f.w2 = weights->w2;
     h->tc_ok = moe::prefill_tc_supported(cfg->hidden, cfg->inter) && moe::prefill_tc_maps(f);
   }
+  if (h->wnorm && (moe::launch_route_norms(w.router_w, E, cfg->hidden, h->wnorm, 0) != cudaSuccess ||
+                   cudaDeviceSynchronize() != cudaSuccess)) {
+    cudaFree(h->ws);
+    delete h;
+    return MOE_ERR_CUDA;
+  }
   *out = h;
   return MOE_OK;
 }
@@ -200,6 +209,7 @@ int moe_route(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* 
   a.x = x; a.Wr = h->w.router_w; a.bias = h->w.router_bias;
   a.logits = h->logits; a.tile_counter = h->tile_counter; a.done_counter = h->done_counter;
   a.ids = topk_ids; a.w = topk_w; a.counts = expert_counts;
+  a.wnorm = h->wnorm; a.err = h->err;
   a.prefetch_shared = T <= MOE_GEMV_MAX_TOKENS;
   a.w13 = h->w.w13; a.w2 = h->w.w2;
   if (h->profiling) h->prof.before(0, stream);
@@ -213,17 +223,24 @@ namespace {
 // The fused decode launch shared by moe_forward (ids given) and moe_decode
 // (routing inside).
 int decode_call(moe_handle h, const uint16_t* x, int T, int route, int32_t* ids, float* w, int32_t* counts,
-                uint16_t* y, const moe_debug* dbg, cudaStream_t stream) {
+                uint16_t* y, const moe_debug* dbg, cudaStream_t stream, float* y32 = nullptr) {
   const moe_config& c = h->cfg;
   moe::DecodeArgs a{};
   a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
+  a.ep_lo = 0;
+  a.ep_hi = c.n_experts;
+  if (h->ep) {
+    a.ep_lo = h->ep_lo;
+    a.ep_hi = h->ep_hi;
+    if (!h->ep_shared) a.n_shared = 0;
+  }
+  a.y32 = y32;
   a.L = 1;
   a.route = route;
   a.layer0 = moe::LayerW{h->w.router_w, h->w.router_bias, h->w.w13, h->w.w2};
   a.x = x;
   a.ids = ids; a.w = w; a.counts = counts;
-  a.logits = h->logits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.tile_cnt = h->tile_cnt;
-  a.yacc = h->yacc; a.err = h->err;
+  a.tlogits = h->tlogits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.err = h->err;
   a.y = y;
   if (dbg) a.dbg = *dbg;
   if (!moe::decode_plan(a, h->n_sms, h->smem_budget)) return MOE_ERR_UNSUPPORTED;
@@ -258,6 +275,7 @@ int moe_forward(moe_handle h, const uint16_t* x, int T, const int32_t* topk_ids,
   if (!h || !x || !topk_ids || !topk_w || !y) return MOE_ERR_ARG;
   if (T < 1 || T > h->max_tokens) return MOE_ERR_ARG;
   if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y)) return MOE_ERR_ALIGN;
+  if (h->ep) return MOE_ERR_UNSUPPORTED;  // a part of a layer: moe_decode_partial
   if (T > MOE_GEMV_MAX_TOKENS) return prefill_call(h, x, T, topk_ids, topk_w, y, dbg, stream);
   return decode_call(h, x, T, 0, const_cast<int32_t*>(topk_ids), const_cast<float*>(topk_w), nullptr, y, dbg,
                      stream);
@@ -270,11 +288,46 @@ int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float*
   if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y) ||
       (expert_counts && !aligned4(expert_counts)))
     return MOE_ERR_ALIGN;
+  if (h->ep) return MOE_ERR_UNSUPPORTED;  // a part of a layer: moe_decode_partial
   if (T > MOE_GEMV_MAX_TOKENS) {
     const int rc = moe_route(h, x, T, topk_ids, topk_w, expert_counts, stream);
     return rc ? rc : prefill_call(h, x, T, topk_ids, topk_w, y, dbg, stream);
   }
   return decode_call(h, x, T, 1, topk_ids, topk_w, expert_counts, y, dbg, stream);
+}
+
+int moe_create_ep(const moe_config* cfg, const moe_weights* local, int max_tokens, int expert_lo, int expert_hi,
+                  int with_shared, moe_handle* out) {
+  if (!cfg || !local || !out) return MOE_ERR_ARG;
+  const int rc0 = validate_config(cfg);
+  if (rc0) return rc0;
+  if (expert_lo < 0 || expert_hi > cfg->n_experts || expert_lo >= expert_hi || max_tokens < 1 ||
+      max_tokens > MOE_GEMV_MAX_TOKENS)
+    return MOE_ERR_ARG;
+  moe_handle h = nullptr;
+  const int rc = moe_create(cfg, local, max_tokens, &h);
+  if (rc) return rc;
+  h->ep = true;
+  h->ep_lo = expert_lo;
+  h->ep_hi = expert_hi;
+  h->ep_shared = with_shared != 0;
+  *out = h;
+  return MOE_OK;
+}
+
+int moe_decode_partial(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float* topk_w,
+                       int32_t* expert_counts, float* y_part, cudaStream_t stream) {
+  if (!h || !x || !topk_ids || !topk_w || !y_part) return MOE_ERR_ARG;
+  if (T < 1 || T > h->max_tokens || T > MOE_GEMV_MAX_TOKENS) return MOE_ERR_ARG;
+  if (!aligned16(x) || !aligned4(topk_ids) || !aligned4(topk_w) || !aligned4(y_part) ||
+      (expert_counts && !aligned4(expert_counts)))
+    return MOE_ERR_ALIGN;
+  return decode_call(h, x, T, 1, topk_ids, topk_w, expert_counts, nullptr, nullptr, stream, y_part);
+}
+
+int moe_round_bf16(const float* v, size_t n, uint16_t* out, cudaStream_t stream) {
+  if ((!v || !out) && n) return MOE_ERR_ARG;
+  return cuda_err(moe::launch_round_bf16(v, n, out, stream));
 }
 
 int moe_device_error(moe_handle h, cudaStream_t stream) {
@@ -287,13 +340,13 @@ int moe_device_error(moe_handle h, cudaStream_t stream) {
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
         cudaMemset(h->amax, 0, static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(h->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
-        cudaMemset(h->tile_cnt, 0, static_cast<size_t>(h->cfg.hidden / 16) * 4) != cudaSuccess ||
-        cudaMemset(h->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.hidden * 8) != cudaSuccess ||
+        // the launch counter restarts at zero: no tagged logit of an earlier launch may match again
+        cudaMemset(h->tlogits, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.n_experts * 8) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   if (e & moe::kErrTimeout) return MOE_ERR_TIMEOUT;
-  if (e & moe::kErrBadId) return MOE_ERR_DEVICE;
+  if (e & (moe::kErrBadId | moe::kErrRouteBound)) return MOE_ERR_DEVICE;
   return MOE_OK;
 }
 
@@ -399,13 +452,11 @@ struct moe_stack_s {
   int max_tokens;
   void* ws;
   moe::LayerW* layers;   // [L] device
-  float* logits;
+  unsigned long long* logits;  // [kMaxTokGemv][E] tagged logits
   float* h;
   unsigned* amax;        // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;
-  unsigned* tile_cnt;
-  double* yacc;
-  uint16_t* ybuf;        // [2][kMaxTokGemv][H]
+  unsigned long long* ty;  // [2][kMaxTokGemv][H/2] tagged y of the stacked layers
   int* err;
   int n_sms;
   int smem_budget;
@@ -435,28 +486,24 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   s->n_sms = layers[0]->n_sms;
   s->smem_budget = layers[0]->smem_budget;
   const size_t n_layers_b = up256(static_cast<size_t>(n_layers) * sizeof(moe::LayerW));
-  const size_t n_logits = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.n_experts * 4);
+  const size_t n_logits = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.n_experts * 8);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * c.inter * 4);
   const size_t n_amax = up256(static_cast<size_t>(n_layers) * moe::kMaxDistinct * moe::kMaxTokGemv * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
-  const size_t n_tcnt = up256(static_cast<size_t>(c.hidden / 16) * 4);
-  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.hidden * 8);
-  const size_t n_ybuf = up256(static_cast<size_t>(2) * moe::kMaxTokGemv * c.hidden * 2);
+  const size_t n_ybuf = up256(static_cast<size_t>(2) * moe::kMaxTokGemv * (c.hidden / 2) * 8);
   const size_t n_err = 256;
-  const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_tcnt + n_yacc + n_ybuf + n_err;
+  const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_ybuf + n_err;
   if (cudaMalloc(&s->ws, bytes) != cudaSuccess) {
     delete s;
     return MOE_ERR_CUDA;
   }
   uint8_t* p = static_cast<uint8_t*>(s->ws);
   s->layers = reinterpret_cast<moe::LayerW*>(p); p += n_layers_b;
-  s->logits = reinterpret_cast<float*>(p); p += n_logits;
+  s->logits = reinterpret_cast<unsigned long long*>(p); p += n_logits;
   s->h = reinterpret_cast<float*>(p); p += n_h;
   s->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
   s->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
-  s->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
-  s->yacc = reinterpret_cast<double*>(p); p += n_yacc;
-  s->ybuf = reinterpret_cast<uint16_t*>(p); p += n_ybuf;
+  s->ty = reinterpret_cast<unsigned long long*>(p); p += n_ybuf;
   s->err = reinterpret_cast<int*>(p);
   moe::LayerW* host = new (std::nothrow) moe::LayerW[n_layers];
   if (!host) {
@@ -495,8 +542,8 @@ int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, in
   a.layers = s->layers;
   a.x = x; a.r_io = r; a.x_io = x; a.eps = eps;
   a.ids = topk_ids; a.w = topk_w;
-  a.logits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync; a.tile_cnt = s->tile_cnt;
-  a.yacc = s->yacc; a.ybuf = s->ybuf; a.err = s->err;
+  a.tlogits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync;
+  a.ty = s->ty; a.err = s->err;
   a.dbg_x = x_layers;
   if (!moe::decode_plan(a, s->n_sms, s->smem_budget)) return MOE_ERR_UNSUPPORTED;
   if (s->profiling) s->prof.before(1, stream);
@@ -514,8 +561,8 @@ int moe_stack_device_error(moe_stack s, cudaStream_t stream) {
     if (cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess ||
         cudaMemset(s->amax, 0, static_cast<size_t>(s->L) * moe::kMaxDistinct * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(s->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
-        cudaMemset(s->tile_cnt, 0, static_cast<size_t>(s->cfg.hidden / 16) * 4) != cudaSuccess ||
-        cudaMemset(s->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.hidden * 8) != cudaSuccess ||
+        cudaMemset(s->logits, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.n_experts * 8) != cudaSuccess ||
+        cudaMemset(s->ty, 0, static_cast<size_t>(2) * moe::kMaxTokGemv * (s->cfg.hidden / 2) * 8) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }

@@ -22,17 +22,15 @@ constexpr int kStaticMaxHidden = 4096;
 constexpr size_t kStaticH = static_cast<size_t>(kMaxDistinct) * kMaxTokGemv * kStaticMaxInter * sizeof(float);
 constexpr size_t kStaticAmax = 1024;     // >= kMaxDistinct * kMaxTokGemv unsigned
 constexpr size_t kStaticSync = 256;      // >= kSyncWords unsigned
-constexpr size_t kStaticTile = (kStaticMaxHidden / 16) * sizeof(unsigned);
-constexpr size_t kStaticYacc = static_cast<size_t>(kMaxTokGemv) * kStaticMaxHidden * sizeof(double);
+constexpr size_t kStaticTlog = static_cast<size_t>(kMaxTokGemv) * MOE_MAX_EXPERTS * sizeof(unsigned long long);
 static_assert(kStaticAmax >= kMaxDistinct * kMaxTokGemv * sizeof(unsigned), "amax area");
 static_assert(kStaticSync >= kSyncWords * sizeof(unsigned), "counter area");
-// layout: h | amax | counters | row-tile counters | float64 accumulators | error
-// word (everything after h starts at zero)
+// layout: h | amax | counters | tagged logits | error word (everything after
+// h starts at zero)
 constexpr size_t kOffAmax = kStaticH;
 constexpr size_t kOffSync = kOffAmax + kStaticAmax;
-constexpr size_t kOffTile = kOffSync + kStaticSync;
-constexpr size_t kOffYacc = kOffTile + kStaticTile;
-constexpr size_t kOffErr = kOffYacc + kStaticYacc;
+constexpr size_t kOffTlog = kOffSync + kStaticSync;
+constexpr size_t kOffErr = kOffTlog + kStaticTlog;
 constexpr size_t kStaticBytes = kOffErr + 256;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
@@ -57,6 +55,12 @@ int scratch_for_current_device(unsigned char** addr, int* n_sms, int* budget) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
         static_smem < 0)
+      return MOE_ERR_CUDA;
+    // the parts that must start at zero; afterwards every call that
+    // completes leaves them zero again, and the error reader clears them
+    // after an error
+    if (cudaMemset(static_cast<unsigned char*>(p) + kOffAmax, 0, kStaticBytes - kOffAmax) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
     g_addr[dev] = static_cast<unsigned char*>(p);
     g_sms[dev] = sms;
@@ -105,12 +109,26 @@ extern "C" int moe_forward_static(const moe_config* cfg, const moe_weights* w, c
   a.h = reinterpret_cast<float*>(base);
   a.amax = reinterpret_cast<unsigned*>(base + kOffAmax);
   a.sync = reinterpret_cast<unsigned*>(base + kOffSync);
-  a.tile_cnt = reinterpret_cast<unsigned*>(base + kOffTile);
-  a.yacc = reinterpret_cast<double*>(base + kOffYacc);
+  a.tlogits = reinterpret_cast<unsigned long long*>(base + kOffTlog);
   a.err = reinterpret_cast<int*>(base + kOffErr);
   a.y = y;
   if (!decode_plan(a, sms, budget)) return MOE_ERR_UNSUPPORTED;
-  // the parts that must start at zero
-  if (cudaMemsetAsync(base + kOffAmax, 0, kStaticBytes - kOffAmax, stream) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_decode(a, sms, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" int moe_forward_static_device_error(cudaStream_t stream) {
+  using namespace moe;
+  unsigned char* base = nullptr;
+  int sms = 0, budget = 0;
+  const int rc = scratch_for_current_device(&base, &sms, &budget);
+  if (rc != MOE_OK) return rc;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int e = 0;
+  if (cudaMemcpy(&e, base + kOffErr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (e && (cudaMemset(base + kOffAmax, 0, kStaticBytes - kOffAmax) != cudaSuccess ||
+            cudaDeviceSynchronize() != cudaSuccess))
+    return MOE_ERR_CUDA;
+  if (e & kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (e & kErrBadId) return MOE_ERR_DEVICE;
+  return MOE_OK;
 }

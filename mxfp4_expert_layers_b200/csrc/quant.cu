@@ -1,6 +1,10 @@
 // Standalone per-row FP8 E4M3 quantisation (the activation step of the W4A8
 // recipe): s = amax / 448, q = E4M3(v / s), round to nearest even with
 // saturation.  One CTA per row.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -39,6 +43,23 @@ quantize_rows_kernel(const float* __restrict__ v, int cols, uint8_t* __restrict_
 cudaError_t launch_quantize_rows(const float* v, int rows, int cols, uint8_t* q, float* s,
                                  cudaStream_t stream) {
   quantize_rows_kernel<<<rows, kThreads, 0, stream>>>(v, cols, q, s);
+  return cudaGetLastError();
+}
+
+namespace {
+
+__global__ void round_bf16_kernel(const float* __restrict__ v, size_t n, uint16_t* __restrict__ out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+}
+
+}  // namespace
+
+cudaError_t launch_round_bf16(const float* v, size_t n, uint16_t* out, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096));
+  round_bf16_kernel<<<blocks, 256, 0, stream>>>(v, n, out);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@ import torch
 import mxfp4_expert_layers_b200 as moe
 import synth
 import synth.gpu
+from oracle import cpp as OC
 from oracle import formats as OF
 from oracle import moe as OM
 
@@ -29,6 +30,27 @@ class LazyExperts(dict):
         v = synth.expert_weights(seed, layer, int(e), H, I)
         self[e] = v
         return v
+
+
+def oracle_layer(host: OM.LayerWeights, x_bits, E, k, I, n_shared=1):
+    """The C++ float64 oracle (bit-equal to oracle.moe.moe_layer, and faster
+    for full-size layers): routes, regenerates the touched experts, runs the
+    experts and the combine."""
+    logits, ids, w = OC.route(x_bits, host.router_w, host.router_bias, k)
+    return oracle_forward(host, x_bits, ids, w, E, I, n_shared, extra={"logits": logits})
+
+
+def oracle_forward(host: OM.LayerWeights, x_bits, ids, w, E, I, n_shared=1, extra=None):
+    """The C++ oracle's experts and combine for given routing (as
+    oracle.moe.moe_forward)."""
+    need = set(np.asarray(ids).ravel().tolist()) | {E + s for s in range(n_shared)}
+    experts = {e: host.experts[e] for e in need}
+    out = OC.forward(x_bits, ids, w, experts, E, I, n_shared)
+    out.update(ids=np.asarray(ids, np.int32), w=np.asarray(w, np.float32),
+               counts=np.bincount(np.asarray(ids).ravel(), minlength=E).astype(np.int32))
+    if extra:
+        out.update(extra)
+    return out
 
 
 def to_dev_u16(a: np.ndarray) -> torch.Tensor:
@@ -144,8 +166,9 @@ def legit_fp8_flip(v_ref: float, code_a: int, code_b: int) -> bool:
 
 
 def check_forward(y_dev, dbg, ref, exact_frac=0.999):
-    """Tolerance of the layer, plus the stronger bit-level checks the exact
-    arithmetic of the GEMV path allows."""
+    """Tolerance of the layer, plus the stronger bit-level checks that the
+    exact arithmetic of the many-token mma.sync kernels (block sums scaled and
+    summed in float64) allows."""
     yg = OF.bf16_to_f64(u16(y_dev))
     yr = OF.bf16_to_f64(ref["y"])
     rel = np.linalg.norm(yg - yr) / max(np.linalg.norm(yr), 1e-300)
@@ -168,8 +191,9 @@ def check_forward(y_dev, dbg, ref, exact_frac=0.999):
     return stats
 
 
-# Tolerance of the tensor-core grouped GEMMs on h.  Their accumulator is
-# float32: each of the K/32 block products (exact) is scaled and added with
+# Tolerance on h of the kernels that accumulate in float32: the decode kernel
+# and the tcgen05 grouped GEMMs.  Each of the K/32 block products (exact) is
+# scaled and added with
 # one rounding of at most 2^-24 of the running sum, so the gate and up sums
 # carry a relative error of order (K/32) * 2^-24 of the sum of their block
 # magnitudes -- about 5e-6 at K = 2560 for sums without cancellation, more

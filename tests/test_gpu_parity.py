@@ -1,9 +1,11 @@
 """GPU parity: the CUDA path through the C ABI against the float64 oracle on
 the same seeded inputs.  Bars: expert ids and counts bit-exact, FP8
 activation bytes bit-exact, BF16 outputs within relative L2 <= 2e-3 and
-max |delta| <= 1e-2 * max |ref|; the GEMV path's exact block arithmetic
-also gives bit-exact FP8 codes of h and (almost always) bit-exact outputs,
-which the tests check too."""
+max |delta| <= 1e-2 * max |ref|.  The decode kernel sums the 32-element
+block products in float32 (tensor core) and the scaled blocks in float32
+(fused multiply-adds), so h is held to the float32-accumulation bound of
+check_forward_tc: within H_TOL_TC of each pair's amax, FP8 codes of h equal
+up to one-step flips at rounding boundaries, and most outputs bit-exact."""
 import numpy as np
 import pytest
 import torch
@@ -13,8 +15,10 @@ import synth
 from oracle import formats as OF
 from oracle import moe as OM
 
-from moe_testlib import (GpuLayer, check_forward, check_route, to_dev, to_dev_u16, u16,
-                         H0, I0)
+from moe_testlib import (GpuLayer, check_forward_tc, check_route, to_dev, to_dev_u16, u16,
+                         H0, I0, REL_L2, MAX_ABS)
+
+check_forward = check_forward_tc  # the decode kernel accumulates in float32
 
 pytestmark = pytest.mark.gpu
 
@@ -209,7 +213,7 @@ def test_gpu_forward_config0_single_token(mode):
             ref = _oracle(L, x)
             check_route(ids, w, counts, ref)
             st = check_forward(y, dbg, ref)
-            assert st["qh_flips"] == 0 and st["h_exact"] == 1.0, st
+            print(mode, step, st)
     finally:
         L.close()
 
@@ -226,13 +230,17 @@ def test_gpu_forward_config1_full_layer(mode):
                 ref = _oracle(L, x)
                 check_route(ids, w, counts, ref)
                 check_forward(y, dbg, ref)
-                # replay: the oracle's down + combine on the GPU's own FP8 h
+                # replay: the oracle's down + combine on the GPU's own FP8 h and
+                # scales isolates the down step: the GPU's output differs from
+                # it only by the float32 sums of 8-block parts
                 qh, sh = dbg["qh"].cpu().numpy()[0], dbg["sh"].cpu().numpy()[0]
                 slots = [(int(e), float(p)) for e, p in zip(ref["ids"][0], ref["w"][0])] + [(512, 1.0)]
                 y64 = np.zeros(H0)
                 for si, (e, p) in enumerate(slots):
                     y64 += p * OM.down_replay(L.host.experts[e], qh[si], sh[si])
-                assert np.array_equal(OF.f64_to_bf16(y64), u16(y)[0])
+                yg = OF.bf16_to_f64(u16(y)[0])
+                assert np.abs(yg - y64).max() <= 2.0 ** -8 * np.abs(y64).max() + 1e-30
+                assert np.mean(OF.f64_to_bf16(y64) == u16(y)[0]) >= 0.99
         finally:
             L.close()
 
@@ -302,6 +310,65 @@ def test_gpu_zero_input_and_zero_weights():
         x = synth.hidden_states(3, 1, 1, H)
         ids, w, counts, y, dbg = _run(L, x)
         assert not (u16(y) & 0x7FFF).any()
+    finally:
+        L.close()
+
+
+def test_gpu_block_sums_beyond_float32_span():
+    """Blocks whose 32 products need more than float32's 24 significant bits:
+    in every 32-element block of x, elements 0..15 are large (FP8 code 448
+    after the per-token scale) and elements 16..31 tiny (E4M3 subnormal
+    codes), against the largest E2M1 magnitude (6) on the large elements and
+    the smallest nonzero one (0.5) on the tiny ones, signs aligned so the
+    large products add up: a block sum near 16 * 6 * 448 = 43008 plus terms of
+    2^-10.  The tensor core's float32 block sum may round there, so this case
+    is held to the layer tolerance and the FP8 rounding-boundary rule on h,
+    not to bit-exact h."""
+    E, H, I, k = 4, 128, 64, 2
+    lw = synth.layer_weights(6, 0, E, H, I)
+    rng = np.random.default_rng(6)
+    big = np.float32(28.0)                      # amax: scale 28 / 448 = 2^-4, code 448
+    x32 = np.empty((2, H), np.float32)
+    for t in range(2):
+        for b in range(H // 32):
+            x32[t, 32 * b:32 * b + 16] = big
+            tiny = (1.0 + rng.integers(0, 8, 16) / 8.0) * 2.0 ** -12 * rng.choice([-1.0, 1.0], 16)
+            x32[t, 32 * b + 16:32 * b + 32] = tiny.astype(np.float32)
+    x = synth._fp32_to_bf16_bits(x32)
+    # gate/up codes: 6 (code 7) on the large elements, +-0.5 (code 1 / 9) on the tiny ones
+    codes = np.empty((E + 1, 2 * I, H), np.uint8)
+    codes[:, :, :] = np.where(rng.random((E + 1, 2 * I, H)) < 0.5, 1, 9)
+    for b in range(H // 32):
+        codes[:, :, 32 * b:32 * b + 16] = 7
+    lw["w13_codes"] = (codes[:, :, 0::2] | (codes[:, :, 1::2] << 4)).astype(np.uint8)
+    L = GpuLayer(6, 0, E, H, I, k=k, weights=lw)
+    try:
+        for mode in MODES:
+            ids, w, counts, y, dbg = _run(L, x, mode=mode)
+            ref = _oracle(L, x)
+            assert np.all(ref["xq"][:, 0::32] == 0x7E)          # the large elements at code 448
+            sub = ref["xq"][:, 16::32] & 0x7F
+            assert np.all((sub > 0) & (sub < 8))                 # the tiny ones subnormal
+            check_route(ids, w, counts, ref)
+            yg, yr = OF.bf16_to_f64(u16(y)), OF.bf16_to_f64(ref["y"])
+            rel = np.linalg.norm(yg - yr) / np.linalg.norm(yr)
+            mx = np.abs(yg - yr).max() / np.abs(yr).max()
+            assert rel <= REL_L2 and mx <= MAX_ABS, (rel, mx)
+            assert np.array_equal(dbg["xq"].cpu().numpy(), ref["xq"])
+            # h within float32 rounding of the block sums; s_h with it
+            hg, hr = dbg["h"].cpu().numpy().astype(np.float64), ref["h"].astype(np.float64)
+            amax = np.abs(hr).max(axis=2, keepdims=True)
+            assert np.all(np.abs(hg - hr) <= 2.0 ** -20 * amax), float((np.abs(hg - hr) / amax).max())
+            assert np.allclose(dbg["sh"].cpu().numpy(), ref["sh"], rtol=2.0 ** -20, atol=0)
+            # each FP8 code of h that differs is one step away, the value near their midpoint
+            qg = dbg["qh"].cpu().numpy()
+            for t, s_, j in np.argwhere(qg != ref["qh"]):
+                va, vb = float(OF.e4m3_value(int(qg[t, s_, j]))), float(OF.e4m3_value(int(ref["qh"][t, s_, j])))
+                v = hr[t, s_, j] / float(ref["sh"][t, s_])
+                assert abs(abs(va) - abs(vb)) <= 2.0 ** -3 * max(abs(va), abs(vb)) + 2.0 ** -9
+                assert abs(v - (va + vb) / 2) <= 2.0 ** -19 * 448 + 1e-6 * abs(v)
+            print(mode, {"rel_l2": rel, "max_rel": mx, "h_exact": float(np.mean(hg == hr)),
+                         "qh_flips": int((qg != ref["qh"]).sum())})
     finally:
         L.close()
 

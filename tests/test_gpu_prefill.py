@@ -16,8 +16,8 @@ import synth
 from oracle import formats as OF
 from oracle import moe as OM
 
-from moe_testlib import (GpuLayer, check_forward, check_forward_tc, check_route, to_dev_u16, u16, H0, REL_L2,
-                         MAX_ABS)
+from moe_testlib import (GpuLayer, check_forward, check_forward_tc, check_route, oracle_forward, to_dev_u16, u16,
+                         H0, REL_L2, MAX_ABS)
 
 KERNELS = {"tc": (moe.MOE_PREFILL_TCGEN05, 3), "exact": (moe.MOE_PREFILL_EXACT, 2)}
 
@@ -108,8 +108,9 @@ def test_gpu_prefill_tc_equals_exact_closely():
 def test_gpu_prefill_config4_sampled():
     """The chunked-prefill workload: 512 tokens through an E = 512 layer with
     the Zipf(1.1) router bias.  Routing of all tokens against the oracle;
-    outputs of 16 sampled tokens against the oracle run on those tokens (each
-    token's output depends on its own routing only)."""
+    outputs against the oracle on 64 sampled tokens plus every token routed
+    to the most popular expert (each token's output depends on its own
+    routing only)."""
     T = 512
     L = GpuLayer(0, 4, 512, bias=True, max_tokens=T)
     try:
@@ -120,9 +121,11 @@ def test_gpu_prefill_config4_sampled():
         assert np.array_equal(counts.cpu().numpy(), rcounts)
         assert np.allclose(w.cpu().numpy(), rw, rtol=1e-6, atol=1e-7)
         assert (rcounts > 0).sum() >= 32  # the skewed routing still touches many experts
+        top = int(np.argmax(rcounts))
         rng = np.random.default_rng(3)
-        sample = np.sort(rng.choice(T, 16, replace=False))
-        ref = OM.moe_forward(x[sample], rids[sample], rw[sample], L.host, 512, L.I, 1)
+        sample = np.union1d(rng.choice(T, 64, replace=False), np.nonzero((rids == top).any(axis=1))[0])
+        assert len(sample) >= 64 + 1 and rcounts[top] > 8, (len(sample), rcounts[top])
+        ref = oracle_forward(L.host, x[sample], rids[sample], rw[sample], 512, L.I, 1)
         yg = OF.bf16_to_f64(u16(y)[sample])
         yr = OF.bf16_to_f64(ref["y"])
         rel = np.linalg.norm(yg - yr) / np.linalg.norm(yr)

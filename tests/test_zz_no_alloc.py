@@ -51,3 +51,26 @@ def test_static_forward_rejects_sizes_beyond_its_array():
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_forward_static(2560, 768, 32, 8, 1, w, 0x1000, 5, 0x1000, 0x1000, 0x1000)
     assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_static_forward_reports_bad_ids():
+    """An expert id outside 0..E-1 is skipped and reported by
+    moe_forward_static_device_error (then cleared); the next call is clean."""
+    E, H, I = 8, 128, 64
+    L = GpuLayer(4, 0, E, H, I, k=2, fill="host")
+    try:
+        x = to_dev_u16(synth.hidden_states(4, 0, 1, H))
+        y = torch.empty((1, H), dtype=torch.int16, device="cuda")
+        w = torch.tensor([[0.75, 0.25]], dtype=torch.float32, device="cuda")
+        bad = torch.tensor([[1, 99]], dtype=torch.int32, device="cuda")
+        moe.moe_forward_static(H, I, E, 2, 1, L.t, x, 1, bad, w, y, torch.cuda.current_stream())
+        assert moe.moe_forward_static_device_error() == moe.MOE_ERR_DEVICE
+        assert moe.moe_forward_static_device_error() == moe.MOE_OK
+        good = torch.tensor([[1, 5]], dtype=torch.int32, device="cuda")
+        moe.moe_forward_static(H, I, E, 2, 1, L.t, x, 1, good, w, y, torch.cuda.current_stream())
+        assert moe.moe_forward_static_device_error() == moe.MOE_OK
+        y_ref, _ = L.forward(x, 1, good, w, debug=False)
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(y), u16(y_ref))
+    finally:
+        L.close()
