@@ -29,9 +29,22 @@ static __device__ unsigned long long g_trace[4][512][64];
       g_trace[k][blockIdx.x + gridDim.x * blockIdx.y][slot] = t_;                   \
     }                                                                               \
   } while (0)
+// Per-warp timestamps (lane 0 of each warp of the first 148 CTAs).
+static __device__ unsigned long long g_wtrace[148][16][16];
+#define MOE_WTRACE(slot)                                                            \
+  do {                                                                              \
+    if ((threadIdx.x & 31) == 0 && blockIdx.x < 148) {                              \
+      unsigned long long t_;                                                        \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                        \
+      g_wtrace[blockIdx.x][threadIdx.x >> 5][(slot) & 15] = t_;                     \
+    }                                                                               \
+  } while (0)
 #else
 #define MOE_TRACE_POINT(k, slot) \
   do {                           \
+  } while (0)
+#define MOE_WTRACE(slot) \
+  do {                   \
   } while (0)
 #endif
 

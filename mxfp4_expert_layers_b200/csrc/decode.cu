@@ -79,7 +79,7 @@ constexpr int kMaxNS = 16;             // ring slots at most
 constexpr int kFeat = 8;               // gate/up features per tile
 constexpr int kBatch = 4;              // blocks whose MMAs are in flight together
 constexpr int kHLoads = 4;             // float4 of h per thread requested at once
-constexpr int kPartBlocks = 8;         // blocks of a down item (K part of a slab)
+constexpr int kPartBlocks = 2;         // blocks of a down item's K part
 constexpr int kMaxDevices = 64;
 
 __host__ __device__ inline size_t up128(size_t v) { return (v + 127) / 128 * 128; }
@@ -289,8 +289,8 @@ __device__ __forceinline__ Work plan_work(const DecodeArgs& a, int nd, int cta, 
   w.nr = rows_of(cta, R, G);
   w.nq = w.nr * nd;
   w.cnt = w.ng + (w.nq + dpe - 1) / dpe;
-  // K parts of kPartBlocks blocks: a fixed split, so a slab's float32 partial
-  // sums do not depend on how many tokens or slabs the call has
+  // K parts of kPartBlocks blocks: a fixed split, so the float32 part sums do
+  // not depend on how many tokens or slabs the call has
   w.dsplit = (a.I / 32 + kPartBlocks - 1) / kPartBlocks;
   return w;
 }
@@ -565,7 +565,6 @@ decode_kernel(DecodeArgs a) {
   float* redp = reinterpret_cast<float*>(smem + a.u_off);          // [ns][4][16][T] gate/up partials
   uint8_t* qh = smem + a.u_off;                                    // [pair][I] permuted E4M3 (down)
   double* yrow = reinterpret_cast<double*>(smem + a.u_off + a.yrow_off);  // [row tile][16][T] (down)
-  const int yrow_len = a.yrow_len;
   // this CTA's router rows (the same in every layer)
   const int row0 = E * cta / G;
   const int nrr = a.route ? E * (cta + 1) / G - row0 : 0;
@@ -801,6 +800,7 @@ decode_kernel(DecodeArgs a) {
           break;
         }
         if (j < 8 && wq == 0) MOE_TRACE_POINT(3, 20 + j);
+        MOE_WTRACE(min(j / kGroups, 3) * 2);
         if (j == first_routed && wq == 0 && lane == 0)
           for (int jd = dn_lo; jd < dn_hi; ++jd) issue_entry(a, rg, lw, dist.expert, wk, jd, ebase + jd);
         const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot;
@@ -808,6 +808,7 @@ decode_kernel(DecodeArgs a) {
         const bool tok = g < T && (dist.mask[u] >> g & 1);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         tile_blocks<kTc>(st, nb, b0, b1, tok ? xq + static_cast<size_t>(g) * H + 8 * t4 : nullptr, acc);
+        MOE_WTRACE(min(j / kGroups, 3) * 2 + 1);
         float* red = redp + static_cast<size_t>(s) * pslot + wq * 16 * T;
         if (2 * t4 < T) {
           red[g * T + 2 * t4] = acc[0];
@@ -907,7 +908,6 @@ decode_kernel(DecodeArgs a) {
         const int u = i / kMaxTokGemv, tt = i % kMaxTokGemv;
         if (pair_of[u][tt] < 0) coef[u][tt] = 0.0;
       }
-      for (int i = tid; i < yrow_len; i += kThreads) yrow[i] = 0.0;
       __syncthreads();  // scales visible
       // FP8 codes of h in the fragment order (each group of 8 elements holds
       // its even elements, then its odd ones); more than kHLoads float4 per
@@ -962,47 +962,59 @@ decode_kernel(DecodeArgs a) {
         }
       }
 
-      // slab items: item it = (slab it / dsplit, K part it % dsplit), warp it mod 16
+      // down items: item it = (row tile it / P, K part it % P), warp it mod
+      // 16; an item runs its K part (kPartBlocks blocks) of every expert's
+      // slab of the row tile, the float32 part sums times w * s_h added in
+      // float64 registers, then leaves its rows in shared memory
       const int g = lane >> 2, t4 = lane & 3;
-      const int ds = wk.dsplit;
-      const int bpp = (nbI + ds - 1) / ds;
-      for (int it = warp; it < nq * ds; it += kWarps) {
-        const int k = it / ds, part = it % ds;
-        const int j = wk.ng + k / rg.dpe, gidx = ebase + j, s = gidx % rg.ns;
-        if (!wait_entry(rg, gidx, a.err, &s_abort)) {
-          if (lane == 0) note_timeout(__LINE__, l, gidx);
-          break;
-        }
-        if (it < 16) MOE_TRACE_POINT(3, 12 + (it >> 2));
-        const int u = k % nd, lr = k / nd;
-        const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot + (k % rg.dpe) * dn_entry_bytes(I);
-        const int pg = g < T ? pair_of[u][g] : -1;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int b0 = min(nbI, part * bpp), b1 = min(nbI, b0 + bpp);
-        tile_blocks<kTc>(st, nbI, b0, b1, pg >= 0 ? qh + static_cast<size_t>(pg) * I + 8 * t4 : nullptr, acc);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          last = atomicAdd(&rg.arr[s], 1) == entry_items(rg, wk, j) - 1;
-          if (last) rg.arr[s] = 0;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last && lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
-        // rows g, g + 8 of tokens 2 t4, 2 t4 + 1, times w * s_h, into the
-        // float64 row sums (every expert of the row tile adds here)
-        double* yr = yrow + static_cast<size_t>(lr) * 16 * T;
-        if (2 * t4 < T) {
-          const double c0 = coef[u][2 * t4];
-          if (c0 != 0.0) {
-            atomicAdd(yr + g * T + 2 * t4, static_cast<double>(acc[0]) * c0);
-            atomicAdd(yr + (g + 8) * T + 2 * t4, static_cast<double>(acc[2]) * c0);
+      const int P = wk.dsplit;
+      for (int it = warp; it < wk.nr * P; it += kWarps) {
+        const int lr = it / P, part = it % P;
+        const int b0 = min(nbI, part * kPartBlocks), b1 = min(nbI, b0 + kPartBlocks);
+        double ya[4] = {0.0, 0.0, 0.0, 0.0};
+        bool good = true;
+        for (int u = 0; u < nd; ++u) {
+          const int k = lr * nd + u;  // slab
+          const int j = wk.ng + k / rg.dpe, gidx = ebase + j, s = gidx % rg.ns;
+          if (!wait_entry(rg, gidx, a.err, &s_abort)) {
+            if (lane == 0) note_timeout(__LINE__, l, gidx);
+            good = false;
+            break;
           }
-          if (!kT1 && 2 * t4 + 1 < T) {
-            const double c1 = coef[u][2 * t4 + 1];
-            if (c1 != 0.0) {
-              atomicAdd(yr + g * T + 2 * t4 + 1, static_cast<double>(acc[1]) * c1);
-              atomicAdd(yr + (g + 8) * T + 2 * t4 + 1, static_cast<double>(acc[3]) * c1);
+          MOE_WTRACE(8 + min(u, 3));
+          const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot + (k % rg.dpe) * dn_entry_bytes(I);
+          const int pg = g < T ? pair_of[u][g] : -1;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          tile_blocks<kTc>(st, nbI, b0, b1, pg >= 0 ? qh + static_cast<size_t>(pg) * I + 8 * t4 : nullptr, acc);
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) {
+            last = atomicAdd(&rg.arr[s], 1) == entry_items(rg, wk, j) - 1;
+            if (last) rg.arr[s] = 0;
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last && lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
+          if (2 * t4 < T) {
+            const double c0 = coef[u][2 * t4];
+            ya[0] = fma(static_cast<double>(acc[0]), c0, ya[0]);
+            ya[2] = fma(static_cast<double>(acc[2]), c0, ya[2]);
+            if (!kT1 && 2 * t4 + 1 < T) {
+              const double c1 = coef[u][2 * t4 + 1];
+              ya[1] = fma(static_cast<double>(acc[1]), c1, ya[1]);
+              ya[3] = fma(static_cast<double>(acc[3]), c1, ya[3]);
             }
+          }
+        }
+        if (!good) break;
+        MOE_WTRACE(12 + min(it / kWarps, 3));
+        // rows g, g + 8 of tokens 2 t4, 2 t4 + 1 of this part: yrow [row tile][part][16][T]
+        double* yp = yrow + (static_cast<size_t>(lr) * P + part) * 16 * T;
+        if (2 * t4 < T) {
+          yp[g * T + 2 * t4] = ya[0];
+          yp[(g + 8) * T + 2 * t4] = ya[2];
+          if (!kT1 && 2 * t4 + 1 < T) {
+            yp[g * T + 2 * t4 + 1] = ya[1];
+            yp[(g + 8) * T + 2 * t4 + 1] = ya[3];
           }
         }
       }
@@ -1010,22 +1022,28 @@ decode_kernel(DecodeArgs a) {
       MOE_TRACE_POINT(3, 10);
       // the CTA's rows of y, each complete: a stacked layer publishes them as
       // tagged words (two rows of one token per word), a plain layer as bf16
+      // the sum over the K parts, in order, of row `row` of token tt
+      auto ysum = [&](int lr, int row, int tt) {
+        double v = 0.0;
+        for (int p = 0; p < P; ++p) v += yrow[((static_cast<size_t>(lr) * P + p) * 16 + row) * T + tt];
+        return v;
+      };
       if (ok && stack) {
         for (int i = tid; i < wk.nr * 8 * T; i += kThreads) {
           const int lr = i / (8 * T), rp = (i / T) % 8, tt = i % T;
-          const double y0 = yrow[(lr * 16 + 2 * rp) * T + tt], y1 = yrow[(lr * 16 + 2 * rp + 1) * T + tt];
+          const double y0 = ysum(lr, 2 * rp, tt), y1 = ysum(lr, 2 * rp + 1, tt);
           st_relaxed_u64(ty_l + (static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + 2 * rp) / 2,
                          ytag | f64_to_bf16_rne(y0) | static_cast<unsigned long long>(f64_to_bf16_rne(y1)) << 16);
         }
       } else if (ok && a.y32) {  // the part of y this call's experts contribute, not yet rounded
         for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
           const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
-          a.y32[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = static_cast<float>(yrow[(lr * 16 + row) * T + tt]);
+          a.y32[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = static_cast<float>(ysum(lr, row, tt));
         }
       } else if (ok) {
         for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
           const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
-          y_l[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = f64_to_bf16_rne(yrow[(lr * 16 + row) * T + tt]);
+          y_l[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = f64_to_bf16_rne(ysum(lr, row, tt));
         }
       }
     }
@@ -1098,6 +1116,9 @@ decode_kernel(DecodeArgs a) {
 extern "C" int moe_trace_read_decode(unsigned long long* out) {
   return cudaMemcpyFromSymbol(out, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -1;
 }
+extern "C" int moe_trace_read_decode_warps(unsigned long long* out) {
+  return cudaMemcpyFromSymbol(out, g_wtrace, sizeof(g_wtrace)) == cudaSuccess ? 0 : -1;
+}
 #endif
 
 cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
@@ -1123,6 +1144,7 @@ cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaS
 bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   const int H = a.H, I = a.I, T = a.T;
   if (T < 1 || T > kMaxTokGemv || n_ctas < 1 || a.L < 1) return false;
+  if (a.ep_lo < 0 || a.ep_hi > a.E || a.ep_lo >= a.ep_hi) return false;  // the routed experts this call runs
   const int R = H / 16;
   const size_t gb = gu_entry_bytes(H), db = dn_entry_bytes(I);
   const size_t slot = up128(gb > db ? gb : db);
@@ -1135,9 +1157,9 @@ bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   // layer start: bf16 x, router partial sums
   a.lpart_off = static_cast<int>(up128(static_cast<size_t>(T) * H * 2));
   const size_t u_start = a.lpart_off + up128(static_cast<size_t>(rr_max) * T * 4 * 8);
-  // down: FP8 h of every pair, the float64 sums of the CTA's row tiles
+  // down: FP8 h of every pair, the float64 sums of the CTA's row tiles per K part
   const int nrt = R / n_ctas + 1;
-  a.yrow_len = nrt * 16 * T;
+  a.yrow_len = nrt * ((I / 32 + kPartBlocks - 1) / kPartBlocks) * 16 * T;
   a.yrow_off = static_cast<int>(up128(static_cast<size_t>(T) * (a.k + a.n_shared) * I));
   const size_t u_down = a.yrow_off + up128(static_cast<size_t>(a.yrow_len) * 8);
   // the most entries one CTA can have in a layer (slots beyond it are unused)

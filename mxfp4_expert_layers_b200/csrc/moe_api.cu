@@ -539,6 +539,8 @@ int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, in
   a.H = c.hidden; a.I = c.inter; a.E = c.n_experts; a.k = c.top_k; a.n_shared = c.n_shared; a.T = T;
   a.L = s->L;
   a.route = 1;
+  a.ep_lo = 0;
+  a.ep_hi = a.E;  // every routed expert
   a.layers = s->layers;
   a.x = x; a.r_io = r; a.x_io = x; a.eps = eps;
   a.ids = topk_ids; a.w = topk_w;

@@ -102,6 +102,8 @@ extern "C" int moe_forward_static(const moe_config* cfg, const moe_weights* w, c
   a.T = T;
   a.L = 1;
   a.route = 0;
+  a.ep_lo = 0;
+  a.ep_hi = a.E;  // every routed expert
   a.layer0 = LayerW{nullptr, nullptr, w->w13, w->w2};
   a.x = x;
   a.ids = const_cast<int32_t*>(topk_ids);
