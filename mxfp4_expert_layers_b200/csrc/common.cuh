@@ -39,7 +39,13 @@ static __device__ unsigned long long g_wtrace[148][16][16];
       g_wtrace[blockIdx.x][threadIdx.x >> 5][(slot) & 15] = t_;                     \
     }                                                                               \
   } while (0)
+// Per-warp cycle counts (lane 0 of each warp of the first 148 CTAs), summed
+// over a launch: [0] gate/up compute, [1] gate/up tiles, [2] down compute,
+// [3] down slabs, [4] gate/up waits, [5] down waits.
+static __device__ long long g_wcyc[148][16][8];
+#define MOE_TR(...) __VA_ARGS__
 #else
+#define MOE_TR(...)
 #define MOE_TRACE_POINT(k, slot) \
   do {                           \
   } while (0)
@@ -292,6 +298,11 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
 }
 __device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Relaxed reduction (max) without a returned value: the issuing warp does
+// not wait for it.
+__device__ __forceinline__ void red_max_u32(unsigned* p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Wait until *p >= target, at most kWaitNs of %globaltimer.  Returns false,

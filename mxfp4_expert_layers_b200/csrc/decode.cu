@@ -71,15 +71,16 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kGroups = 4;             // gate/up warp groups
-constexpr int kQuarters = kWarps / kGroups;  // warps per tile (K quarters)
+constexpr int kWarps = 7;                 // compute warps (the K parts of tiles and slabs)
+constexpr int kProducer = kWarps;         // the warp that requests the weight copies
+constexpr int kAllWarps = kWarps + 1;
+constexpr int kThreads = 32 * kAllWarps;  // 256: 255 registers a thread, no local memory
 constexpr int kMaxNS = 16;             // ring slots at most
 constexpr int kFeat = 8;               // gate/up features per tile
 constexpr int kBatch = 4;              // blocks whose MMAs are in flight together
-constexpr int kHLoads = 4;             // float4 of h per thread requested at once
-constexpr int kPartBlocks = 2;         // blocks of a down item's K part
+constexpr int kHLoads = 7;             // float4 of h per thread requested at once (9 pairs x 768 in one round)
+constexpr int kRnU = 3;                // y units a thread requests together (residual add)
+constexpr int kDnPB = 5;               // blocks of a warp's K part of a down slab, at most (I <= 1120)
 constexpr int kMaxDevices = 64;
 
 __host__ __device__ inline size_t up128(size_t v) { return (v + 127) / 128 * 128; }
@@ -226,27 +227,14 @@ __device__ __noinline__ void note_timeout(int line, int layer, int entry) {
 #endif
 }
 
-// Output row tiles (16 rows of y) of CTA c: whole tiles, R / G each and one
-// more for the last R mod G CTAs.  A CTA owns every expert's slab of its row
-// tiles, so each y row is summed and rounded by one CTA.
-__device__ __forceinline__ int rows_of(int c, int R, int G) { return R / G + (c >= G - R % G ? 1 : 0); }
-__device__ __forceinline__ int row0_of(int c, int R, int G) { return (R / G) * c + max(0, c - (G - R % G)); }
-
-// First gate/up tile of CTA c (c = G: the tile count).  The layer's bytes
-// (gate/up tiles and down slabs) are shared out evenly: a CTA's gate/up
-// quota is what its down slabs leave of an even share, and the tiles are
-// given out in proportion to the quotas (integer arithmetic, so every CTA
-// computes the same boundaries).  A CTA's tiles are consecutive.
-__device__ __forceinline__ int gstart_of(int c, int G, int R, int nd, int ntiles, long long gb, long long db) {
-  const long long W = static_cast<long long>(ntiles) * gb + static_cast<long long>(R) * nd * db;
-  const int base = R / G, extra = R % G;
-  // G x (even share - down bytes), for CTAs with base and base + 1 row tiles
-  const long long qa = max(0LL, W - static_cast<long long>(G) * base * nd * db);
-  const long long qb = max(0LL, W - static_cast<long long>(G) * (base + 1) * nd * db);
-  const int nb = max(0, c - (G - extra));  // CTAs before c with base + 1 row tiles
-  const long long P = static_cast<long long>(c - nb) * qa + static_cast<long long>(nb) * qb;
-  const long long PG = static_cast<long long>(G - extra) * qa + static_cast<long long>(extra) * qb;
-  return PG > 0 ? static_cast<int>((P * ntiles + PG / 2) / PG) : 0;
+// Even split of n units over G CTAs: the first unit of CTA c (c = G: n).
+__device__ __forceinline__ int split_at(int n, int c, int G) {
+  return static_cast<int>(static_cast<long long>(n) * c / G);
+}
+// The CTA whose share holds unit s (the last CTA whose first unit is <= s;
+// never a CTA with an empty share).
+__device__ __forceinline__ int owner_of(int n, int s, int G) {
+  return static_cast<int>((static_cast<long long>(s + 1) * G - 1) / n);
 }
 
 __device__ __forceinline__ LayerW layer_ptrs(const DecodeArgs& a, int l) {
@@ -269,81 +257,81 @@ struct Ring {
   int ns, slot, dpe;
 };
 
-// What one layer asks of this CTA (the same values in every thread).
+// What one layer asks of this CTA (the same values in every thread).  The
+// gate/up tiles and the down slabs are each split evenly over the CTAs.
 struct Work {
   int nd;          // distinct experts of the call
   int g0, ng;      // gate/up tiles g0 .. g0+ng-1 (tile i: features 8 (i mod I/8) of distinct expert i / (I/8))
-  int r0, nr;      // output row tiles r0 .. r0+nr-1
-  int nq;          // down slabs nr * nd: slab k = row tile r0 + k / nd of distinct expert k mod nd
-  int cnt;         // entries: ng tiles, then ceil(nq / dpe) slab groups
-  int dsplit;      // down items per slab (K parts)
+  int s0, nq;      // down slabs s0 .. s0+nq-1 (slab s: output row tile s / nd of distinct expert s mod nd)
+  int cnt;         // entries: ng tiles, then the slabs dpe to an entry
 };
 
 __device__ __forceinline__ Work plan_work(const DecodeArgs& a, int nd, int cta, int G, int dpe) {
   Work w;
-  const int cpe = a.I / kFeat, R = a.H / 16, ntiles = nd * cpe;
+  const int ntiles = nd * (a.I / kFeat), nslab = nd * (a.H / 16);
   w.nd = nd;
-  w.g0 = gstart_of(cta, G, R, nd, ntiles, gu_entry_bytes(a.H), dn_entry_bytes(a.I));
-  w.ng = gstart_of(cta + 1, G, R, nd, ntiles, gu_entry_bytes(a.H), dn_entry_bytes(a.I)) - w.g0;
-  w.r0 = row0_of(cta, R, G);
-  w.nr = rows_of(cta, R, G);
-  w.nq = w.nr * nd;
+  w.g0 = split_at(ntiles, cta, G);
+  w.ng = split_at(ntiles, cta + 1, G) - w.g0;
+  w.s0 = split_at(nslab, cta, G);
+  w.nq = split_at(nslab, cta + 1, G) - w.s0;
   w.cnt = w.ng + (w.nq + dpe - 1) / dpe;
-  // K parts of kPartBlocks blocks: a fixed split, so the float32 part sums do
-  // not depend on how many tokens or slabs the call has
-  w.dsplit = (a.I / 32 + kPartBlocks - 1) / kPartBlocks;
   return w;
 }
+
+// Everything issue_entry needs besides the entry, in shared memory (one
+// copy per CTA; thread 0 points w13 / w2 at the layer whose entries are
+// being requested).  Kept out of registers: the requests are issued from
+// inside the gate/up and down loops.
+struct IssueCtx {
+  const uint8_t* w13;  // packed gate/up tiles of the layer
+  const uint8_t* w2;   // packed down slabs of the layer
+  uint8_t* ring;       // slot 0 of the weight ring
+  uint64_t* full;      // [ns] mbarriers
+  int* iss;            // [ns] entries issued into each slot so far
+  int slot, ns, dpe, H, I, E, ep_lo, ep_hi;
+};
 
 // Position of expert e (routed < E, shared E + s) in the weight arrays: the
 // arrays hold the routed experts ep_lo .. ep_hi-1 (all of them unless the
 // layer is split over several GPUs), then the shared experts.
-__device__ __forceinline__ int weight_index(const DecodeArgs& a, int e) {
-  return e < a.E ? e - a.ep_lo : (a.ep_hi - a.ep_lo) + (e - a.E);
+__device__ __forceinline__ int weight_index(const IssueCtx* c, int e) {
+  return e < c->E ? e - c->ep_lo : (c->ep_hi - c->ep_lo) + (e - c->E);
 }
 
 // Request entry j of the layer (launch-wide entry gidx) into its slot.
 // `expert` maps distinct-expert positions to expert indices.
-__device__ __forceinline__ void issue_entry(const DecodeArgs& a, const Ring& rg, const LayerW& lw, const int* expert,
-                                            const Work& wk, int j, int gidx) {
-  const int s = gidx % rg.ns;
-  uint8_t* dst = rg.base + static_cast<size_t>(s) * rg.slot;
-  if (j < wk.ng) {
-    const int cpe = a.I / kFeat, i = wk.g0 + j, bytes = gu_entry_bytes(a.H);
-    mbar_expect_tx(&rg.full[s], static_cast<uint32_t>(bytes));
-    bulk_g2s(dst, lw.w13 + (static_cast<size_t>(weight_index(a, expert[i / cpe])) * cpe + i % cpe) * bytes,
-             static_cast<uint32_t>(bytes), &rg.full[s]);
+__device__ __noinline__ void issue_entry(const IssueCtx* c, const int* expert, const Work* wk, int j, int gidx) {
+  const int s = gidx % c->ns;
+  uint8_t* dst = c->ring + static_cast<size_t>(s) * c->slot;
+  if (j < wk->ng) {
+    const int cpe = c->I / kFeat, i = wk->g0 + j, bytes = gu_entry_bytes(c->H);
+    mbar_expect_tx(&c->full[s], static_cast<uint32_t>(bytes));
+    bulk_g2s(dst, c->w13 + (static_cast<size_t>(weight_index(c, expert[i / cpe])) * cpe + i % cpe) * bytes,
+             static_cast<uint32_t>(bytes), &c->full[s]);
   } else {
-    const int d = j - wk.ng, ka = d * rg.dpe, n = min(rg.dpe, wk.nq - ka);
-    const int bytes = dn_entry_bytes(a.I);
-    mbar_expect_tx(&rg.full[s], static_cast<uint32_t>(n * bytes));
-    for (int k = ka; k < ka + n; ++k)
+    const int d = j - wk->ng, ka = d * c->dpe, n = min(c->dpe, wk->nq - ka);
+    const int bytes = dn_entry_bytes(c->I), R = c->H / 16;
+    mbar_expect_tx(&c->full[s], static_cast<uint32_t>(n * bytes));
+    for (int k = ka; k < ka + n; ++k) {
+      const int sl = wk->s0 + k;
       bulk_g2s(dst + (k - ka) * bytes,
-               lw.w2 + (static_cast<size_t>(weight_index(a, expert[k % wk.nd])) * (a.H / 16) + wk.r0 + k / wk.nd) * bytes,
-               static_cast<uint32_t>(bytes), &rg.full[s]);
+               c->w2 + (static_cast<size_t>(weight_index(c, expert[sl % wk->nd])) * R + sl / wk->nd) * bytes,
+               static_cast<uint32_t>(bytes), &c->full[s]);
+    }
   }
-  atomicAdd(&rg.iss[s], 1);
-}
-
-// Items of entry j (the consumers that must count themselves in before the
-// slot is free again).
-__device__ __forceinline__ int entry_items(const Ring& rg, const Work& wk, int j) {
-  if (j < wk.ng) return kQuarters;
-  const int d = j - wk.ng;
-  return min(rg.dpe, wk.nq - d * rg.dpe) * wk.dsplit;
+  atomicAdd(&c->iss[s], 1);
 }
 
 // Wait until entry gidx has landed in its slot: first until it has been
 // issued (the slot's previous entry consumed), then for its bytes.  Bounded;
 // gives up early when another warp raised the abort flag.
-__device__ __noinline__ bool wait_entry_slow(const Ring& rg, int gidx, int* err, int* abort) {
-  const int s = gidx % rg.ns, use = gidx / rg.ns;
-  const volatile int* is = rg.iss + s;
+__device__ __noinline__ bool wait_entry_slow(const int* iss, uint64_t* full, int s, int use, int* err, int* abort) {
+  const volatile int* is = iss + s;
   const volatile int* ab = abort;
   const unsigned long long t0 = global_ns();
   for (long long i = 1; i < kSpinLimit; ++i) {
     if (*is <= use) __nanosleep(64);  // not issued yet: the slot's previous entry is in use
-    else if (mbar_try_wait_sleep(&rg.full[s], use & 1, 1000u)) return true;
+    else if (mbar_try_wait_sleep(&full[s], use & 1, 1000u)) return true;
     if ((i & 15) == 0) {
       if (*ab) return false;
       if (global_ns() - t0 > kWaitNs) break;
@@ -353,75 +341,123 @@ __device__ __noinline__ bool wait_entry_slow(const Ring& rg, int gidx, int* err,
   *reinterpret_cast<volatile int*>(abort) = 1;
   return false;
 }
+// (the ring's fields go by value: a reference would put the ring in local
+// memory, and local memory misses the small L1 that the shared-memory
+// carve-out leaves)
 __device__ __forceinline__ bool wait_entry(const Ring& rg, int gidx, int* err, int* abort) {
   const int s = gidx % rg.ns, use = gidx / rg.ns;
   if (*reinterpret_cast<const volatile int*>(rg.iss + s) > use && mbar_try_wait(&rg.full[s], use & 1)) return true;
-  return wait_entry_slow(rg, gidx, err, abort);
+  return wait_entry_slow(rg.iss, rg.full, s, use, err, abort);
 }
 
-// 8 bfloat16 y values (chunk u of [T][H]) from the tagged words of a layer's
-// y (two values per 64-bit word, tag in the high half): read until all four
-// words carry `tag`.  Bounded; false (kErrTimeout) when a word never arrives.
-__device__ __forceinline__ bool load_y8(const unsigned long long* ty, int u, unsigned tag, uint4& out, int* err,
-                                        const int* abort) {
-  const unsigned long long* p = ty + 4 * static_cast<size_t>(u);
-  unsigned long long v[4];
+// Waits until the shared counter *p reaches target (one thread).  Bounded;
+// false (kErrTimeout and the abort flag) when it does not.
+__device__ __noinline__ bool wait_count(const int* p, int target, int* err, int* abort) {
+  const volatile int* vp = p;
+  const unsigned long long t0 = global_ns();
+  for (long long i = 0; i < kSpinLimit; ++i) {
+    if (*vp >= target) {
+      __threadfence_block();
+      return true;
+    }
+    if ((i & 15) == 15) {
+      if (*reinterpret_cast<const volatile int*>(abort)) return false;
+      if (global_ns() - t0 > kWaitNs) break;
+    }
+    __nanosleep(20);
+  }
+  atomicOr(err, kErrTimeout);
+  *reinterpret_cast<volatile int*>(abort) = 1;
+  return false;
+}
+
+// Partial sums of a layer's y for the output row tiles shared by several
+// CTAs: each contributor other than the last publishes its float64 sum of
+// its slabs as two 64-bit words (low, high 32 bits of the value, each |
+// tag << 32) at [tile][k][token][row], k = the CTA's index minus the tile's
+// first contributing CTA; the last contributor (the finisher) adds them in
+// CTA order before its own sum and writes y.
+__host__ __device__ inline size_t ypart_index(int r, int k, int tt, int row, int ypk, int T) {
+  return (((static_cast<size_t>(r) * ypk + k) * T + tt) * 16 + row) * 2;
+}
+
+// Waits until 4 consecutive tagged words (32-bit payload | tag << 32) all
+// carry `tag`; v holds the words already read and receives the current ones.
+// Bounded; false (kErrTimeout) when a word never arrives.
+__device__ __forceinline__ bool poll_words4(const unsigned long long* p, unsigned tag, unsigned long long (&v)[4],
+                                        int* err, const int* abort) {
   const unsigned long long t0 = global_ns();
   for (long long it = 0;; ++it) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = ld_relaxed_u64(p + j);
     bool ok = true;
 #pragma unroll
     for (int j = 0; j < 4; ++j) ok &= static_cast<unsigned>(v[j] >> 32) == tag;
-    if (ok) break;
+    if (ok) return true;
     if ((it & 7) == 7 && (global_ns() - t0 > kWaitNs || it > kSpinLimit ||
                           *reinterpret_cast<const volatile int*>(abort))) {
       atomicOr(err, kErrTimeout);
       return false;
     }
     __nanosleep(32);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = ld_relaxed_u64(p + j);
   }
-  out = make_uint4(static_cast<unsigned>(v[0]), static_cast<unsigned>(v[1]), static_cast<unsigned>(v[2]),
-                   static_cast<unsigned>(v[3]));
-  return true;
 }
 
 // Residual add and RMS normalisation of the stack (every CTA, same values):
-// r = bf16(r + y); x = bf16(r / sqrt(mean(r^2) + eps)), float64 arithmetic.
+// r = bf16(r + y), x = bf16(r / sqrt(mean(r^2) + eps)), float64 arithmetic.
 // rs and xb are [T][H] bfloat16 in shared memory; y comes from the tagged
-// words of the previous layer (every CTA's rows, read as they arrive).
-// Returns false when a wait gave up (the caller aborts).
-__device__ bool residual_norm(const DecodeArgs& a, uint16_t* rs, const unsigned long long* ty, unsigned tag,
-                              uint16_t* xb, double (*red)[kMaxTokGemv], double* den_s, int* abort) {
-  const int H = a.H, T = a.T, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int upr = H / 8;
+// words of the previous layer (every row tile's finisher writes them).  A
+// thread requests the words of kRnU chunks together (one round trip once
+// they have arrived).  Returns false when a wait gave up (the caller aborts).
+__device__ __forceinline__ bool residual_norm(int H, int T, float eps, int* err, uint16_t* rs,
+                                              const unsigned long long* ty, const unsigned* ycount,
+                                              unsigned ytarget, uint16_t* xb, double (*red)[kMaxTokGemv],
+                                              double* den_s, int* abort) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int upr = H / 8, nu = T * upr;
   double ss[kMaxTokGemv] = {0.0, 0.0, 0.0, 0.0};
   bool good = true;
-  for (int u = tid; u < T * upr && good; u += kThreads) {
-    uint4 yv;
-    good = load_y8(ty, u, tag, yv, a.err, abort);
-    const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
-    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-    uint32_t o[4];
-    double part = 0.0;
+  // every row tile's finisher counts its tiles in after writing their y
+  // words; once the count is complete the words are read once (polling the
+  // words themselves instead costs the CTAs that start polling first)
+  if (tid == 0 && !poll_geq_bounded(ycount, ytarget, err)) *reinterpret_cast<volatile int*>(abort) = 1;
+  if (!__syncthreads_and(*reinterpret_cast<volatile int*>(abort) == 0)) return false;
+  for (int u0 = tid; u0 < nu; u0 += kThreads * kRnU) {
+    unsigned long long v[kRnU][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float r0, r1, y0, y1;
-      bf16x2_f32(rw[j], r0, r1);
-      bf16x2_f32(yw[j], y0, y1);
-      const uint16_t s0 = f64_to_bf16_rne(static_cast<double>(r0) + static_cast<double>(y0));
-      const uint16_t s1 = f64_to_bf16_rne(static_cast<double>(r1) + static_cast<double>(y1));
-      o[j] = static_cast<uint32_t>(s0) | (static_cast<uint32_t>(s1) << 16);
-      const double q0 = bf16_bits_to_f32(s0), q1 = bf16_bits_to_f32(s1);
-      part = fma(q0, q0, part);
-      part = fma(q1, q1, part);
+    for (int i = 0; i < kRnU; ++i) {
+      const int u = u0 + i * kThreads;
+      if (u < nu) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[i][j] = __ldcg(ty + 4 * static_cast<size_t>(u) + j);
+      }
     }
-    reinterpret_cast<uint4*>(rs)[u] = make_uint4(o[0], o[1], o[2], o[3]);
-    const int t = u / upr;
 #pragma unroll
-    for (int tt = 0; tt < kMaxTokGemv; ++tt)
-      if (tt == t) ss[tt] += part;
+    for (int i = 0; i < kRnU; ++i) {
+      const int u = u0 + i * kThreads;
+      if (u >= nu) continue;
+      const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
+      const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+      uint32_t o[4];
+      double part = 0.0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float r0, r1, y0, y1;
+        bf16x2_f32(rw[j], r0, r1);
+        bf16x2_f32(static_cast<uint32_t>(v[i][j]), y0, y1);
+        const uint16_t s0 = f64_to_bf16_rne(static_cast<double>(r0) + static_cast<double>(y0));
+        const uint16_t s1 = f64_to_bf16_rne(static_cast<double>(r1) + static_cast<double>(y1));
+        o[j] = static_cast<uint32_t>(s0) | (static_cast<uint32_t>(s1) << 16);
+        const double q0 = bf16_bits_to_f32(s0), q1 = bf16_bits_to_f32(s1);
+        part = fma(q0, q0, part);
+        part = fma(q1, q1, part);
+      }
+      reinterpret_cast<uint4*>(rs)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+      const int tt = u / upr;
+#pragma unroll
+      for (int t = 0; t < kMaxTokGemv; ++t)
+        if (t == tt) ss[t] += part;
+    }
   }
 #pragma unroll
   for (int tt = 0; tt < kMaxTokGemv; ++tt) {
@@ -434,16 +470,16 @@ __device__ bool residual_norm(const DecodeArgs& a, uint16_t* rs, const unsigned 
   }
   if (tid < T) {
     double s = 0.0;
-    for (int w = 0; w < kWarps; ++w) s += red[w][tid];
-    den_s[tid] = sqrt(s / static_cast<double>(H) + static_cast<double>(a.eps));
+    for (int w = 0; w < kAllWarps; ++w) s += red[w][tid];
+    den_s[tid] = sqrt(s / static_cast<double>(H) + static_cast<double>(eps));
   }
   __syncthreads();
-  for (int u = tid; u < T * upr; u += kThreads) {
+  for (int u = tid; u < nu; u += kThreads) {
     const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
     const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
     const double den = den_s[u / upr];
     uint32_t o[4];
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < 4; ++j) {
       float r0, r1;
       bf16x2_f32(rw[j], r0, r1);
@@ -466,8 +502,9 @@ __device__ __forceinline__ float block_scale(uint32_t e8) { return __uint_as_flo
 // mma.sync m16n8k32 (A = the E2M1 codes widened to E4M3 bytes holding
 // value * 2^-6, B = the FP8 activations of tokens 0..T-1 as columns) gives
 // the float32 block sums (exact when the 32 products span at most 24 bits),
-// scaled by 2^(E-121) and summed in float32 (fused multiply-adds).  acc: rows
-// g and g+8 of tokens 2*t4 and 2*t4+1 (lane = 4g + t4).  `xbp` points at this
+// scaled by 2^(E-121) and summed in float32 (fused multiply-adds), kBatch
+// blocks in flight at a time (the last batch predicated).  acc: rows g and
+// g+8 of tokens 2*t4 and 2*t4+1 (lane = 4g + t4).  `xbp` points at this
 // lane's activation bytes of block 0 (nullptr: a zero column).
 template <int kT>
 __device__ __forceinline__ void tile_blocks(const uint8_t* st, int nb, int b0, int b1, const uint8_t* xbp,
@@ -475,46 +512,31 @@ __device__ __forceinline__ void tile_blocks(const uint8_t* st, int nb, int b0, i
   const int lane = threadIdx.x & 31, g = lane >> 2;
   const uint8_t* cp = st + 8 * lane;
   const uint8_t* sp = st + 256 * nb + 2 * g;
-  int b = b0;
-  // whole batches: no per-block bounds
-  for (; b + kBatch <= b1; b += kBatch) {
+  for (int b = b0; b < b1; b += kBatch) {
     float d[kBatch][4];
     uint32_t sc[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const uint2 cw = *reinterpret_cast<const uint2*>(cp + 256 * (b + u));
-      sc[u] = *reinterpret_cast<const uint16_t*>(sp + 16 * (b + u));
-      const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
-      uint2 q = make_uint2(0u, 0u);
-      if (xbp) q = *reinterpret_cast<const uint2*>(xbp + 32 * (b + u));
-      mma_fp8(d[u], af, q.x, q.y);
+      if (b + u < b1) {
+        const uint2 cw = *reinterpret_cast<const uint2*>(cp + 256 * (b + u));
+        sc[u] = *reinterpret_cast<const uint16_t*>(sp + 16 * (b + u));
+        const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+        uint2 q = make_uint2(0u, 0u);
+        if (xbp) q = *reinterpret_cast<const uint2*>(xbp + 32 * (b + u));
+        mma_fp8(d[u], af, q.x, q.y);
+      }
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const float sa = block_scale(sc[u] & 0xFFu), sb = block_scale(sc[u] >> 8);
-      acc[0] = fmaf(d[u][0], sa, acc[0]);
-      acc[2] = fmaf(d[u][2], sb, acc[2]);
-      if (kT > 1) {
-        acc[1] = fmaf(d[u][1], sa, acc[1]);
-        acc[3] = fmaf(d[u][3], sb, acc[3]);
+      if (b + u < b1) {
+        const float sa = block_scale(sc[u] & 0xFFu), sb = block_scale(sc[u] >> 8);
+        acc[0] = fmaf(d[u][0], sa, acc[0]);
+        acc[2] = fmaf(d[u][2], sb, acc[2]);
+        if (kT > 1) {
+          acc[1] = fmaf(d[u][1], sa, acc[1]);
+          acc[3] = fmaf(d[u][3], sb, acc[3]);
+        }
       }
-    }
-  }
-  // the remaining blocks one at a time
-  for (; b < b1; ++b) {
-    float d[4];
-    const uint2 cw = *reinterpret_cast<const uint2*>(cp + 256 * b);
-    const uint32_t sc = *reinterpret_cast<const uint16_t*>(sp + 16 * b);
-    const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
-    uint2 q = make_uint2(0u, 0u);
-    if (xbp) q = *reinterpret_cast<const uint2*>(xbp + 32 * b);
-    mma_fp8(d, af, q.x, q.y);
-    const float sa = block_scale(sc & 0xFFu), sb = block_scale(sc >> 8);
-    acc[0] = fmaf(d[0], sa, acc[0]);
-    acc[2] = fmaf(d[2], sb, acc[2]);
-    if (kT > 1) {
-      acc[1] = fmaf(d[1], sa, acc[1]);
-      acc[3] = fmaf(d[3], sb, acc[3]);
     }
   }
 }
@@ -529,6 +551,8 @@ decode_kernel(DecodeArgs a) {
   __shared__ __align__(8) uint64_t full[kMaxNS];
   __shared__ __align__(8) uint64_t fr;
   __shared__ int iss[kMaxNS], arr[kMaxNS];
+  __shared__ int parr[2 * kMaxNS];  // part sums written into each gate/up partial area so far
+  __shared__ int freed[kMaxNS];     // entries of each slot consumed so far
   __shared__ int s_riss;  // router-row copies issued
   __shared__ Distinct dist;
   __shared__ int s_pre_expert[MOE_MAX_SHARED];
@@ -541,17 +565,19 @@ decode_kernel(DecodeArgs a) {
   __shared__ int s_ids[kMaxTokGemv * MOE_MAX_TOPK];
   __shared__ float s_w[kMaxTokGemv * MOE_MAX_TOPK];
   __shared__ float xs[kMaxTokGemv];
-  __shared__ float red_f[kWarps][kMaxTokGemv];
-  __shared__ double red_d[kWarps][kMaxTokGemv];
+  __shared__ float red_f[kAllWarps][kMaxTokGemv];
+  __shared__ double red_d[kAllWarps][kMaxTokGemv];
   __shared__ double den_s[kMaxTokGemv];
   __shared__ int s_abort;
   __shared__ int s_flag;
   __shared__ int s_hist[MOE_MAX_EXPERTS];
+  __shared__ IssueCtx ictx;
+  __shared__ Work s_wk, s_pw;          // this layer's work; the predicted work of the first layer
+  __shared__ LayerW s_lay, s_lay_next;  // this layer's and the next layer's weights
 
   constexpr int kTc = kT1 ? 1 : 2;  // accumulator columns per lane
   const int H = a.H, I = a.I, T = kT1 ? 1 : a.T, E = a.E, S = a.n_shared, L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = warp / kQuarters, wq = warp % kQuarters;
   const int G = gridDim.x, cta = blockIdx.x;
   const int cpe = I / kFeat;
   const int nb = H / 32, nbI = I / 32;
@@ -562,45 +588,68 @@ decode_kernel(DecodeArgs a) {
   uint16_t* rs = reinterpret_cast<uint16_t*>(smem + a.rs_off);     // [T][H] bf16 residual (stack)
   uint16_t* xb = reinterpret_cast<uint16_t*>(smem + a.u_off);      // [T][H] bf16 x (layer start)
   double* lpart = reinterpret_cast<double*>(smem + a.u_off + a.lpart_off);  // router partial sums
-  float* redp = reinterpret_cast<float*>(smem + a.u_off);          // [ns][4][16][T] gate/up partials
+  float* redp = reinterpret_cast<float*>(smem + a.u_off);          // [2 ns][warp][16][T] gate/up partials
   uint8_t* qh = smem + a.u_off;                                    // [pair][I] permuted E4M3 (down)
-  double* yrow = reinterpret_cast<double*>(smem + a.u_off + a.yrow_off);  // [row tile][16][T] (down)
+  double* yrow = reinterpret_cast<double*>(smem + a.u_off + a.yrow_off);  // [row tile][warp][16][T] (down)
   // this CTA's router rows (the same in every layer)
   const int row0 = E * cta / G;
   const int nrr = a.route ? E * (cta + 1) / G - row0 : 0;
   // One token routed by this kernel always has k + S distinct experts, so
-  // the next layer's work split is known in advance and its first entries --
-  // gate/up tiles of the shared experts, the first tiles of every layer -- can
-  // be requested before its routing.
+  // the first layer's work split is known in advance and its first entries
+  // -- gate/up tiles of the shared experts, the first tiles of every layer --
+  // are requested before the dependency wait (later layers request theirs
+  // after routing: copies in flight would slow the polls of the exchanges).
   const bool predict = a.route && T == 1 && a.ep_lo == 0 && a.ep_hi == E;
-  Work pw{};
-  int npre = 0;  // entries of the coming layer already requested
+  int npre = 0;  // entries of the first layer already requested
+  int pnd = 0;   // distinct experts of the predicted work
   if (predict) {
-    pw = plan_work(a, min(a.k, E) + S, cta, G, a.dpe);
+    const Work pw = plan_work(a, min(a.k, E) + S, cta, G, a.dpe);
     npre = max(0, min(min(pw.g0 + pw.ng, S * cpe) - pw.g0, a.ns));
+    pnd = pw.nd;
+    if (tid == 0) s_pw = pw;
   }
 
   MOE_TRACE_POINT(3, 0);
+  MOE_TR(if (tid == 0) {
+    unsigned sm_;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm_));
+    g_trace[3][cta][13] = sm_;
+  })
+  MOE_TR(long long cyc[8] = {0, 0, 0, 0, 0, 0, 0, 0};)
+  // (traced builds: the phase stamps of the last layer only)
+#define MOE_TRACE_LAYER(k, slot) \
+  do {                           \
+    if (l == L - 1) MOE_TRACE_POINT(k, slot); \
+  } while (0)
   // ---- before the dependency wait: the first layer's router rows and
   // shared-expert tiles (weights only)
-  LayerW lw = layer_ptrs(a, 0);
   if (tid < kMaxNS) { iss[tid] = 0; arr[tid] = 0; }
+  if (tid < 2 * kMaxNS) parr[tid] = 0;
+  if (tid < kMaxNS) freed[tid] = 0;
   if (tid == 0) {
     for (int s = 0; s < a.ns; ++s) mbar_init(&full[s], 1);
     mbar_init(&fr, 1);
     fence_mbar_init();
     s_riss = 0;
     s_abort = 0;
+    s_lay = layer_ptrs(a, 0);
+    ictx = IssueCtx{s_lay.w13, s_lay.w2, smem, full, iss, a.slot_bytes, a.ns, a.dpe, H, I, E, a.ep_lo, a.ep_hi};
   }
   if (tid < MOE_MAX_SHARED) s_pre_expert[tid] = E + tid;
   __syncthreads();
-  if (tid == 0 && nrr > 0) {
-    mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
-    bulk_g2s(rr, lw.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
-    s_riss = 1;
+  // (every weight copy is requested by one thread, lane 0 of the producer
+  // warp: a copy request waits while the copy engine's queue is full, and
+  // that wait must not hold up the warps that compute)
+  if (warp == kProducer && lane == 0) {
+    if (nrr > 0) {
+      mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
+      bulk_g2s(rr, s_lay.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
+      s_riss = 1;
+    }
+    for (int j = 0; j < npre; ++j) issue_entry(&ictx, s_pre_expert, &s_pw, j, j);
   }
-  if (warp < npre && lane == 0) issue_entry(a, rg, lw, s_pre_expert, pw, warp, warp);
   int ebase = 0;  // launch-wide number of this layer's entry 0
+  int gbase = 0;  // launch-wide number of this layer's gate/up tile 0
 
   pdl_wait();
   pdl_trigger();
@@ -609,8 +658,10 @@ decode_kernel(DecodeArgs a) {
   // last CTA counted itself in before this one could start), layer
   const unsigned tag0 = __ldcg(a.sync + kSyncEpoch) * 256u + 1u;
 
-  for (int l = 0; l < L && ok; ++l) {
-    MOE_TRACE_POINT(3, 1);
+  // (a stack runs one pass more, l = L: the residual and normalisation
+  // after its last layer, then leaves the loop)
+  for (int l = 0; l < L + (kStack ? 1 : 0) && ok; ++l) {
+    MOE_TRACE_LAYER(3, 1);
     // ---- 1. input x
     if (l == 0) {
       for (int u = tid; u < T * H / 8; u += kThreads) {
@@ -620,13 +671,22 @@ decode_kernel(DecodeArgs a) {
       __syncthreads();
     } else if (kStack) {
       // the previous layer's y: every CTA's rows, read as their tagged words arrive
-      if (!residual_norm(a, rs, a.ty + static_cast<size_t>((l - 1) & 1) * T * H / 2, tag0 + (l - 1), xb, red_d,
-                         den_s, &s_abort)) {
+      if (!residual_norm(H, T, a.eps, a.err, rs, a.ty + static_cast<size_t>((l - 1) & 1) * T * H / 2,
+                         a.sync + kSyncY, static_cast<unsigned>(l * (H / 16)), xb, red_d, den_s, &s_abort)) {
         ok = false;
         note_timeout(__LINE__, l, -1);
         break;
       }
+      if (l == L) {  // after the last layer: CTA 0 writes the residual and x
+        if (cta == 0)
+          for (int u = tid; u < T * H / 8; u += kThreads) {
+            reinterpret_cast<uint4*>(a.r_io)[u] = reinterpret_cast<const uint4*>(rs)[u];
+            reinterpret_cast<uint4*>(a.x_io)[u] = reinterpret_cast<const uint4*>(xb)[u];
+          }
+        break;
+      }
     }
+    MOE_TRACE_LAYER(3, 12);
     if (kDebug && a.dbg_x && cta == 0)
       for (int u = tid; u < T * H / 8; u += kThreads)
         reinterpret_cast<uint4*>(a.dbg_x + static_cast<size_t>(l) * T * H)[u] = reinterpret_cast<const uint4*>(xb)[u];
@@ -653,7 +713,7 @@ decode_kernel(DecodeArgs a) {
       __syncthreads();
       if (tid < T) {
         float amax = 0.f;
-        for (int i = 0; i < kWarps; ++i) amax = fmaxf(amax, red_f[i][tid]);
+        for (int i = 0; i < kAllWarps; ++i) amax = fmaxf(amax, red_f[i][tid]);
         xs[tid] = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
         if (kDebug && cta == 0 && a.dbg.xs) a.dbg.xs[tid] = xs[tid];
       }
@@ -676,12 +736,12 @@ decode_kernel(DecodeArgs a) {
                                                              q[4] | q[5] << 8 | q[6] << 16 | q[7] << 24);
       }
     }
-    MOE_TRACE_POINT(3, 2);
+    MOE_TRACE_LAYER(3, 2);
 
     // ---- 2. routing
     int32_t* ids_l = a.ids ? a.ids + static_cast<size_t>(l) * T * a.k : nullptr;
     float* w_l = a.w ? a.w + static_cast<size_t>(l) * T * a.k : nullptr;
-    const LayerW lw_next = l + 1 < L ? layer_ptrs(a, l + 1) : lw;
+    if (tid == 0) s_lay_next = l + 1 < L ? layer_ptrs(a, l + 1) : s_lay;
     if (a.route) {
       if (nrr > 0 && !mbar_wait_bounded(&fr, l & 1, a.err)) {
         ok = false;
@@ -690,7 +750,7 @@ decode_kernel(DecodeArgs a) {
       const uint16_t* rrows = reinterpret_cast<const uint16_t*>(rr);
       const int ql = H / 4;  // elements per quarter row
       const int items = ok ? nrr * T * 4 : 0;
-      for (int it = warp; it < items; it += kWarps) {
+      for (int it = warp; it < items; it += kAllWarps) {
         const int ri = it / (T * 4), tt = (it / 4) % T, qq = it % 4;
         const uint4* wrow = reinterpret_cast<const uint4*>(rrows + static_cast<size_t>(ri) * H + qq * ql);
         const uint4* xrow = reinterpret_cast<const uint4*>(xb + static_cast<size_t>(tt) * H + qq * ql);
@@ -705,18 +765,12 @@ decode_kernel(DecodeArgs a) {
         const int ri = i / T, tt = i % T;
         const double* p = lpart + (ri * T + tt) * 4;
         float lg = static_cast<float>((p[0] + p[1]) + (p[2] + p[3]));
-        if (lw.bias) lg = __fadd_rn(lg, __ldg(lw.bias + row0 + ri));
+        if (s_lay.bias) lg = __fadd_rn(lg, __ldg(s_lay.bias + row0 + ri));
         st_relaxed_u64(a.tlogits + static_cast<size_t>(tt) * E + row0 + ri,
                        static_cast<unsigned long long>(tag) << 32 | __float_as_uint(lg));
       }
       __syncthreads();
-      MOE_TRACE_POINT(3, 3);
-      // the router rows are used: the next layer's stream in meanwhile
-      if (tid == 0 && l + 1 < L && nrr > 0 && ok) {
-        mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
-        bulk_g2s(rr, lw_next.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
-        ++s_riss;
-      }
+      MOE_TRACE_LAYER(3, 3);
       if (warp < T && ok &&
           !topk_warp(a.tlogits + static_cast<size_t>(warp) * E, tag, E, a.k, s_ids + warp * a.k, s_w + warp * a.k,
                      a.err, &s_abort)) {
@@ -725,7 +779,7 @@ decode_kernel(DecodeArgs a) {
       }
       ok = __syncthreads_and(ok);
       if (!ok) break;
-      MOE_TRACE_POINT(3, 4);
+      MOE_TRACE_LAYER(3, 4);
       if (cta == 0) {
         if (tid < T * a.k) {
           if (ids_l) ids_l[tid] = s_ids[tid];
@@ -745,11 +799,13 @@ decode_kernel(DecodeArgs a) {
     }
     if (warp == 0) build_distinct(s_ids, s_w, T, a.k, E, S, dist, wsum, a.err, cta == 0 && !a.route, a.ep_lo, a.ep_hi);
     __syncthreads();
-    MOE_TRACE_POINT(3, 5);
+    MOE_TRACE_LAYER(3, 5);
 
     // ---- this layer's work and its first entries (warp w issues entries w, w + 16, ...)
     const Work wk = plan_work(a, dist.n, cta, G, rg.dpe);
-    if (predict && wk.nd != pw.nd) {  // the requested entries would not be this layer's (never for routed T = 1)
+    if (tid == 0) s_wk = wk;
+    __syncthreads();
+    if (npre > 0 && wk.nd != pnd) {  // the requested entries would not be this layer's (never for routed T = 1)
       if (tid == 0) atomicOr(a.err, kErrTimeout);
       ok = false;
       break;
@@ -760,11 +816,6 @@ decode_kernel(DecodeArgs a) {
     // bytes are needed only after the gate/up barrier)
     const int first_routed = wk.ng > 0 && wk.g0 + wk.ng > S * cpe ? max(0, S * cpe - wk.g0) : -1;
     const int dn_lo = max(wk.ng, npre), dn_hi = min(wk.cnt, rg.ns);
-    if (lane == 0) {
-      for (int j = npre + warp; j < min(wk.ng, rg.ns); j += kWarps) issue_entry(a, rg, lw, dist.expert, wk, j, ebase + j);
-      if (first_routed < 0)
-        for (int j = dn_lo + warp; j < dn_hi; j += kWarps) issue_entry(a, rg, lw, dist.expert, wk, j, ebase + j);
-    }
     // pair table of the down step (off the critical path): the (expert,
     // token) pairs in order, numbered by a ballot prefix count
     if (warp == kWarps - 1) {
@@ -783,33 +834,57 @@ decode_kernel(DecodeArgs a) {
       }
       if (lane == 0) s_npairs = base_p;
     }
-    MOE_TRACE_POINT(3, 6);
+    MOE_TRACE_LAYER(3, 6);
 
-    // ---- 3. gate/up + SwiGLU: group grp takes tiles grp, grp + 4, ...; warp
-    // wq of the group the K quarter wq of each
-    {
+    // ---- 3. gate/up + SwiGLU: warp w takes the K part w of every tile
+    // (blocks w nb / W .. (w + 1) nb / W, W warps), so all warps work on the tile
+    // that landed first
+    if (warp == kProducer) {
+      // the producer: the layer's first entries, then each entry whose slot
+      // held a gate/up tile as soon as that tile is consumed
+      if (lane == 0) {
+        bool pok = true;
+        for (int j = npre; j < min(wk.ng, rg.ns); ++j) issue_entry(&ictx, dist.expert, &s_wk, j, ebase + j);
+        if (dn_lo < dn_hi) {
+          if (first_routed >= 0) pok = wait_entry(rg, ebase + first_routed, a.err, &s_abort);
+          for (int j = dn_lo; j < dn_hi && pok; ++j) issue_entry(&ictx, dist.expert, &s_wk, j, ebase + j);
+        }
+        for (int n = rg.ns; n < wk.cnt && n - rg.ns < wk.ng && pok; ++n) {
+          const int gi = ebase + n;
+          pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
+          if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
+        }
+      }
+      __syncwarp();
+    } else {
       const int g = lane >> 2, t4 = lane & 3;
-      const int nbq = (nb + kQuarters - 1) / kQuarters;
-      const int b0 = min(nb, wq * nbq), b1 = min(nb, b0 + nbq);
+      const int b0 = warp * nb / kWarps, b1 = (warp + 1) * nb / kWarps;
       unsigned* amax_l = a.amax + static_cast<size_t>(l) * kMaxDistinct * kMaxTokGemv;
-      const int pslot = kQuarters * 16 * T;  // partial sums per slot
-      for (int j = grp; j < wk.ng; j += kGroups) {
+      const int pslot = kWarps * 16 * T;  // partial sums per slot
+      for (int j = 0; j < wk.ng; ++j) {
         const int gidx = ebase + j, s = gidx % rg.ns;
+        MOE_TR(long long c0 = clock64();)
         if (!wait_entry(rg, gidx, a.err, &s_abort)) {
           if (lane == 0) note_timeout(__LINE__, l, gidx);
           break;
         }
-        if (j < 8 && wq == 0) MOE_TRACE_POINT(3, 20 + j);
-        MOE_WTRACE(min(j / kGroups, 3) * 2);
-        if (j == first_routed && wq == 0 && lane == 0)
-          for (int jd = dn_lo; jd < dn_hi; ++jd) issue_entry(a, rg, lw, dist.expert, wk, jd, ebase + jd);
+        MOE_TR(cyc[4] += clock64() - c0;)
+        if (j < 8 && warp == 0) MOE_TRACE_LAYER(3, 20 + j);
+        MOE_WTRACE(min(j, 3) * 2);
         const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot;
         const int i = wk.g0 + j, u = i / cpe, f0 = (i % cpe) * kFeat;
         const bool tok = g < T && (dist.mask[u] >> g & 1);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        MOE_TR(c0 = clock64();)
         tile_blocks<kTc>(st, nb, b0, b1, tok ? xq + static_cast<size_t>(g) * H + 8 * t4 : nullptr, acc);
-        MOE_WTRACE(min(j / kGroups, 3) * 2 + 1);
-        float* red = redp + static_cast<size_t>(s) * pslot + wq * 16 * T;
+        MOE_TR(cyc[0] += clock64() - c0; cyc[1] += 1;)
+        MOE_WTRACE(min(j, 3) * 2 + 1);
+        // this warp's part sums go to partial area pa, by the launch-wide
+        // gate/up tile number gt (2 ns areas: a warp may start on tile gt + ns
+        // before the epilogue of tile gt has read them, but not on gt + 2 ns,
+        // whose weights need a slot that the epilogue's warp frees after it)
+        const int gt = gbase + j, pa = gt % (2 * rg.ns), puse = gt / (2 * rg.ns);
+        float* red = redp + static_cast<size_t>(pa) * pslot + warp * 16 * T;
         if (2 * t4 < T) {
           red[g * T + 2 * t4] = acc[0];
           red[(g + 8) * T + 2 * t4] = acc[2];
@@ -819,45 +894,49 @@ decode_kernel(DecodeArgs a) {
           }
         }
         __syncwarp();
-        int last = 0;
         if (lane == 0) {
           __threadfence_block();
-          last = atomicAdd(&rg.arr[s], 1) == kQuarters - 1;
-          if (last) rg.arr[s] = 0;
-          __threadfence_block();
+          atomicAdd(&parr[pa], 1);
+          // the last warp done with the slot's weights frees it (the producer
+          // requests its next entry)
+          if (atomicAdd(&rg.arr[s], 1) == kWarps - 1) {
+            rg.arr[s] = 0;
+            __threadfence_block();
+            atomicAdd(&freed[s], 1);
+          }
         }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
+        // the epilogue of tile j: warp j mod W, once every warp's part sums
+        // are in (a rotating warp, so that no warp does it for every tile)
+        if (warp != j % kWarps) continue;
+        if (lane == 0 && !wait_count(&parr[pa], kWarps * (puse + 1), a.err, &s_abort)) note_timeout(__LINE__, l, gidx);
         __syncwarp();  // lane 0's acquire orders the other lanes' reads too
-        if (j < 8) MOE_TRACE_POINT(3, 28 + j);
-        // the 4 quarters' sums of feature f, token tt (lanes o = f * T + tt)
-        const float* rs4 = redp + static_cast<size_t>(s) * pslot;
+        if (j < 8) MOE_TRACE_LAYER(3, 28 + j);
+        // the parts' sums of feature f, token tt (lanes o = f * T + tt), in part order
+        const float* rs4 = redp + static_cast<size_t>(pa) * pslot;
         double gs = 0.0, us = 0.0;
         const int f = lane / T, tt = lane % T;
         if (lane < kFeat * T) {
-#pragma unroll
-          for (int q = 0; q < kQuarters; ++q) {
+#pragma unroll 4
+          for (int q = 0; q < kWarps; ++q) {
             gs += rs4[(q * 16 + f) * T + tt];
             us += rs4[(q * 16 + f + 8) * T + tt];
           }
         }
-        __syncwarp();
-        // the slot is free: its next entry streams in while SwiGLU runs
-        if (lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
         if (lane < kFeat * T && (dist.mask[u] >> tt & 1)) {
-          const double gv = static_cast<double>(xs[tt]) * gs;
-          const double uv = static_cast<double>(xs[tt]) * us;
-          const float hv = static_cast<float>(gv / (1.0 + exp(-gv)) * uv);
+          // SwiGLU in float32 (a short dependency chain)
+          const float gv = static_cast<float>(static_cast<double>(xs[tt]) * gs);
+          const float uv = static_cast<float>(static_cast<double>(xs[tt]) * us);
+          const float hv = gv / (1.0f + expf(-gv)) * uv;
           __stcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + f0 + f, hv);
           const float m = fabsf(hv);
-          if (m > 0.f) atomicMax(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
+          if (m > 0.f) red_max_u32(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
         }
-        if (j < 8) MOE_TRACE_POINT(3, 40 + j);
+        if (j < 8) MOE_TRACE_LAYER(3, 40 + j);
       }
     }
     ok = __syncthreads_and(!s_abort);
     if (!ok) break;
-    MOE_TRACE_POINT(3, 7);
+    MOE_TRACE_LAYER(3, 7);
     // every CTA's h and amax are needed by every CTA's down slabs
     if (tid == 0) {
       __threadfence();
@@ -869,15 +948,25 @@ decode_kernel(DecodeArgs a) {
     }
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    MOE_TRACE_POINT(3, 8);
+    MOE_TRACE_LAYER(3, 8);
 
     // ---- 4. down + combine
-    // y of this layer: a plain layer's output (bf16), or a stacked layer's
-    // tagged words (two rows per word) that the next layer polls
-    uint16_t* y_l = a.y;
+    // the next layer's router rows stream in while the down slabs are
+    // summed (requested then rather than earlier: a burst of copies in
+    // flight slows the polls and loads of the exchanges before it)
+    auto prefetch_router = [&]() {  // (lane 0 of the producer)
+      if (a.route && l + 1 < L && nrr > 0) {
+        mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
+        bulk_g2s(rr, s_lay_next.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
+        ++s_riss;
+      }
+    };
+    // this layer's partial words and (stack) y words; a stack alternates two areas
+    unsigned long long* yp_l = a.ypart + static_cast<size_t>(l & 1) * (H / 16) * a.ypk * T * 16 * 2;
     unsigned long long* ty_l = a.ty ? a.ty + static_cast<size_t>(l & 1) * T * H / 2 : nullptr;
-    const unsigned long long ytag = static_cast<unsigned long long>(tag0 + l) << 32;
+    const unsigned ytag = tag0 + static_cast<unsigned>(l);
     const int nd = wk.nd, nq = wk.nq;
+    int nfin = 0;  // row tiles this CTA finishes (writes y of)
     if (nq > 0) {
       const int np = s_npairs;
       unsigned* amax_l = a.amax + static_cast<size_t>(l) * kMaxDistinct * kMaxTokGemv;
@@ -940,11 +1029,11 @@ decode_kernel(DecodeArgs a) {
         }
       }
       __syncthreads();
-      MOE_TRACE_POINT(3, 9);
+      MOE_TRACE_LAYER(3, 9);
       // debug copies by the CTA holding row tile 0 (every CTA with down work has all of qh)
-      if (kDebug && wk.r0 == 0 && (a.dbg.qh || a.dbg.h || a.dbg.sh)) {
+      if (kDebug && wk.s0 == 0 && (a.dbg.qh || a.dbg.h || a.dbg.sh)) {
         const int Sl = a.k + S;
-        for (int pp = warp; pp < T * Sl; pp += kWarps) {
+        for (int pp = warp; pp < T * Sl; pp += kAllWarps) {
           const int tt = pp / Sl, si = pp % Sl;
           const int e = si < a.k ? s_ids[tt * a.k + si] : E + (si - a.k);
           int u = -1;
@@ -962,129 +1051,214 @@ decode_kernel(DecodeArgs a) {
         }
       }
 
-      // down items: item it = (row tile it / P, K part it % P), warp it mod
-      // 16; an item runs its K part (kPartBlocks blocks) of every expert's
-      // slab of the row tile, the float32 part sums times w * s_h added in
-      // float64 registers, then leaves its rows in shared memory
+      // down: warp w takes the K part w of every slab of the CTA (blocks
+      // w nbI / W .. (w + 1) nbI / W, W warps), slabs in order; the float32
+      // part sums times w * s_h are added in float64 registers per output
+      // row tile and left in shared memory ([tile][warp][16][T]) when the
+      // slabs move to the next row tile
       const int g = lane >> 2, t4 = lane & 3;
-      const int P = wk.dsplit;
-      for (int it = warp; it < wk.nr * P; it += kWarps) {
-        const int lr = it / P, part = it % P;
-        const int b0 = min(nbI, part * kPartBlocks), b1 = min(nbI, b0 + kPartBlocks);
-        double ya[4] = {0.0, 0.0, 0.0, 0.0};
-        bool good = true;
-        for (int u = 0; u < nd; ++u) {
-          const int k = lr * nd + u;  // slab
-          const int j = wk.ng + k / rg.dpe, gidx = ebase + j, s = gidx % rg.ns;
-          if (!wait_entry(rg, gidx, a.err, &s_abort)) {
-            if (lane == 0) note_timeout(__LINE__, l, gidx);
-            good = false;
-            break;
+      const int b0 = warp * nbI / kWarps, nbp = (warp + 1) * nbI / kWarps - b0;
+      const int db = dn_entry_bytes(I);
+      const int r_first = wk.s0 / nd;
+      int sr = r_first, su = wk.s0 - r_first * nd;  // row tile and distinct expert of the next slab
+      double ya[4] = {0.0, 0.0, 0.0, 0.0};
+      int cur = r_first;
+      auto flush = [&](int r) {
+        double* yq = yrow + (static_cast<size_t>(r - r_first) * kWarps + warp) * 16 * T;
+        if (2 * t4 < T) {
+          yq[g * T + 2 * t4] = ya[0];
+          yq[(g + 8) * T + 2 * t4] = ya[2];
+          if (!kT1 && 2 * t4 + 1 < T) {
+            yq[g * T + 2 * t4 + 1] = ya[1];
+            yq[(g + 8) * T + 2 * t4 + 1] = ya[3];
           }
-          MOE_WTRACE(8 + min(u, 3));
-          const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot + (k % rg.dpe) * dn_entry_bytes(I);
-          const int pg = g < T ? pair_of[u][g] : -1;
+        }
+        ya[0] = ya[1] = ya[2] = ya[3] = 0.0;
+      };
+      const int ndn = (nq + rg.dpe - 1) / rg.dpe;
+      if (warp == kProducer) {
+        // the producer: each entry whose slot held a down entry as soon as
+        // that is consumed; then the next layer's router rows
+        if (lane == 0) {
+          bool pok = true;
+          for (int n = max(rg.ns, wk.ng + rg.ns); n < wk.cnt && pok; ++n) {
+            const int gi = ebase + n;
+            pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
+            if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
+          }
+          prefetch_router();
+        }
+        __syncwarp();
+      } else {
+      bool good = true;
+      for (int e = 0; e < ndn && good; ++e) {
+        const int j = wk.ng + e, gidx = ebase + j, s = gidx % rg.ns;
+        MOE_TR(long long c0 = clock64();)
+        if (!wait_entry(rg, gidx, a.err, &s_abort)) {
+          if (lane == 0) note_timeout(__LINE__, l, gidx);
+          good = false;
+          break;
+        }
+        MOE_TR(cyc[5] += clock64() - c0; c0 = clock64();)
+        MOE_WTRACE(8 + min(e, 3));
+        const uint8_t* se = rg.base + static_cast<size_t>(s) * rg.slot;
+        const int ka = e * rg.dpe, n = min(rg.dpe, nq - ka);
+        for (int k = 0; k < n; ++k) {
+          // slab wk.s0 + ka + k: row tile sr, distinct expert su
+          const int pg = g < T ? pair_of[su][g] : -1;
+          const uint8_t* st = se + k * db;
+          float d[kDnPB][4];
+          uint32_t sc[kDnPB];
+#pragma unroll
+          for (int bb = 0; bb < kDnPB; ++bb) {
+            if (bb < nbp) {
+              const int blk = b0 + bb;
+              const uint2 cw = *reinterpret_cast<const uint2*>(st + 8 * lane + 256 * blk);
+              sc[bb] = *reinterpret_cast<const uint16_t*>(st + 256 * nbI + 2 * g + 16 * blk);
+              const uint32_t af[4] = {e4m3_lo(cw.x), e4m3_lo(cw.y), e4m3_hi(cw.x), e4m3_hi(cw.y)};
+              uint2 q = make_uint2(0u, 0u);
+              if (pg >= 0) q = *reinterpret_cast<const uint2*>(qh + static_cast<size_t>(pg) * I + 8 * t4 + 32 * blk);
+              mma_fp8(d[bb], af, q.x, q.y);
+            }
+          }
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          tile_blocks<kTc>(st, nbI, b0, b1, pg >= 0 ? qh + static_cast<size_t>(pg) * I + 8 * t4 : nullptr, acc);
-          __syncwarp();
-          int last = 0;
-          if (lane == 0) {
-            last = atomicAdd(&rg.arr[s], 1) == entry_items(rg, wk, j) - 1;
-            if (last) rg.arr[s] = 0;
+#pragma unroll
+          for (int bb = 0; bb < kDnPB; ++bb) {
+            if (bb < nbp) {
+              const float sa = block_scale(sc[bb] & 0xFFu), sb = block_scale(sc[bb] >> 8);
+              acc[0] = fmaf(d[bb][0], sa, acc[0]);
+              acc[2] = fmaf(d[bb][2], sb, acc[2]);
+              if (!kT1) {
+                acc[1] = fmaf(d[bb][1], sa, acc[1]);
+                acc[3] = fmaf(d[bb][3], sb, acc[3]);
+              }
+            }
           }
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (last && lane == 0 && j + rg.ns < wk.cnt) issue_entry(a, rg, lw, dist.expert, wk, j + rg.ns, gidx + rg.ns);
+          if (sr != cur) {
+            flush(cur);
+            cur = sr;
+          }
           if (2 * t4 < T) {
-            const double c0 = coef[u][2 * t4];
+            const double c0 = coef[su][2 * t4];
             ya[0] = fma(static_cast<double>(acc[0]), c0, ya[0]);
             ya[2] = fma(static_cast<double>(acc[2]), c0, ya[2]);
             if (!kT1 && 2 * t4 + 1 < T) {
-              const double c1 = coef[u][2 * t4 + 1];
+              const double c1 = coef[su][2 * t4 + 1];
               ya[1] = fma(static_cast<double>(acc[1]), c1, ya[1]);
               ya[3] = fma(static_cast<double>(acc[3]), c1, ya[3]);
             }
           }
-        }
-        if (!good) break;
-        MOE_WTRACE(12 + min(it / kWarps, 3));
-        // rows g, g + 8 of tokens 2 t4, 2 t4 + 1 of this part: yrow [row tile][part][16][T]
-        double* yp = yrow + (static_cast<size_t>(lr) * P + part) * 16 * T;
-        if (2 * t4 < T) {
-          yp[g * T + 2 * t4] = ya[0];
-          yp[(g + 8) * T + 2 * t4] = ya[2];
-          if (!kT1 && 2 * t4 + 1 < T) {
-            yp[g * T + 2 * t4 + 1] = ya[1];
-            yp[(g + 8) * T + 2 * t4 + 1] = ya[3];
+          if (++su == nd) {
+            su = 0;
+            ++sr;
           }
         }
+        MOE_TR(cyc[2] += clock64() - c0; cyc[3] += n;)
+        // this warp is done with the entry; the last warp frees the slot
+        __syncwarp();
+        if (lane == 0 && atomicAdd(&rg.arr[s], 1) == kWarps - 1) {
+          rg.arr[s] = 0;
+          __threadfence_block();
+          atomicAdd(&freed[s], 1);
+        }
       }
+      if (good) flush(cur);
+      }
+      MOE_WTRACE(12);
       ok = __syncthreads_and(!s_abort);
-      MOE_TRACE_POINT(3, 10);
-      // the CTA's rows of y, each complete: a stacked layer publishes them as
-      // tagged words (two rows of one token per word), a plain layer as bf16
-      // the sum over the K parts, in order, of row `row` of token tt
-      auto ysum = [&](int lr, int row, int tt) {
+      MOE_TRACE_LAYER(3, 10);
+      // the CTA's sum of row tile r_first + rl, row, token tt: its warps' parts in order
+      auto ysum = [&](int rl, int row, int tt) {
         double v = 0.0;
-        for (int p = 0; p < P; ++p) v += yrow[((static_cast<size_t>(lr) * P + p) * 16 + row) * T + tt];
+        const double* yq = yrow + static_cast<size_t>(rl) * kWarps * 16 * T + row * T + tt;
+#pragma unroll 4
+        for (int w = 0; w < kWarps; ++w) v += yq[w * 16 * T];
         return v;
       };
-      if (ok && stack) {
-        for (int i = tid; i < wk.nr * 8 * T; i += kThreads) {
-          const int lr = i / (8 * T), rp = (i / T) % 8, tt = i % T;
-          const double y0 = ysum(lr, 2 * rp, tt), y1 = ysum(lr, 2 * rp + 1, tt);
-          st_relaxed_u64(ty_l + (static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + 2 * rp) / 2,
-                         ytag | f64_to_bf16_rne(y0) | static_cast<unsigned long long>(f64_to_bf16_rne(y1)) << 16);
+      // Output, two rows of a token at a time.  The CTA's sum of a row tile
+      // it holds whole is y.  For a tile shared with other CTAs, all but the
+      // last of them (the finisher) publish their sums as partial words, and
+      // the finisher adds them, in CTA order, before its own sum.  y goes to
+      // the caller (bf16, or float32 for a part of a layer split over GPUs)
+      // or, in a stack, to the tagged words the next layer reads.
+      const int nslab = nd * (H / 16);
+      const int ntl = (wk.s0 + nq - 1) / nd - r_first + 1;
+      for (int rl = 0; rl < ntl; ++rl) nfin += owner_of(nslab, (r_first + rl) * nd + nd - 1, G) == cta;
+      for (int i = tid; i < ntl * 8 * T && ok; i += kThreads) {
+        const int rl = i / (8 * T), row = 2 * ((i / T) % 8), tt = i % T, r = r_first + rl;
+        const double v0 = ysum(rl, row, tt), v1 = ysum(rl, row + 1, tt);
+        const int c0 = owner_of(nslab, r * nd, G), c1 = owner_of(nslab, r * nd + nd - 1, G);
+        const unsigned long long tg = static_cast<unsigned long long>(ytag) << 32;
+        if (cta != c1) {
+          unsigned long long* wp = yp_l + ypart_index(r, cta - c0, tt, row, a.ypk, T);
+          const unsigned long long b0v = static_cast<unsigned long long>(__double_as_longlong(v0));
+          const unsigned long long b1v = static_cast<unsigned long long>(__double_as_longlong(v1));
+          st_relaxed_u64(wp + 0, tg | (b0v & 0xFFFFFFFFull));
+          st_relaxed_u64(wp + 1, tg | (b0v >> 32));
+          st_relaxed_u64(wp + 2, tg | (b1v & 0xFFFFFFFFull));
+          st_relaxed_u64(wp + 3, tg | (b1v >> 32));
+          continue;
         }
-      } else if (ok && a.y32) {  // the part of y this call's experts contribute, not yet rounded
-        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
-          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
-          a.y32[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = static_cast<float>(ysum(lr, row, tt));
+        double o0 = 0.0, o1 = 0.0;  // the other contributors' sums, in CTA order
+        for (int c = c0; c < c1 && ok; ++c) {
+          if (split_at(nslab, c + 1, G) == split_at(nslab, c, G)) continue;  // an empty share
+          const unsigned long long* wp = yp_l + ypart_index(r, c - c0, tt, row, a.ypk, T);
+          unsigned long long w4[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w4[j] = ld_relaxed_u64(wp + j);
+          ok = poll_words4(wp, ytag, w4, a.err, &s_abort);
+          o0 += __longlong_as_double(static_cast<long long>((w4[1] << 32) | (w4[0] & 0xFFFFFFFFull)));
+          o1 += __longlong_as_double(static_cast<long long>((w4[3] << 32) | (w4[2] & 0xFFFFFFFFull)));
         }
-      } else if (ok) {
-        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
-          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
-          y_l[static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row] = f64_to_bf16_rne(ysum(lr, row, tt));
+        const double y0 = o0 + v0, y1 = o1 + v1;
+        const size_t yi = static_cast<size_t>(tt) * H + 16 * r + row;
+        if (stack) {
+          st_relaxed_u64(ty_l + yi / 2, tg | f64_to_bf16_rne(y0) | static_cast<unsigned long long>(f64_to_bf16_rne(y1)) << 16);
+        } else if (a.y32) {
+          a.y32[yi] = static_cast<float>(y0);
+          a.y32[yi + 1] = static_cast<float>(y1);
+        } else {
+          a.y[yi] = f64_to_bf16_rne(y0);
+          a.y[yi + 1] = f64_to_bf16_rne(y1);
         }
+      }
+      if (!ok) {
+        if (tid == 0) *reinterpret_cast<volatile int*>(&s_abort) = 1;
       }
     }
-    if (nq == 0 && wk.nr > 0 && ok) {
+    if (nq == 0 && warp == kProducer && lane == 0) prefetch_router();
+    if (nd == 0 && !stack && ok) {
       // no expert of this call contributes (every id skipped and no shared
-      // expert): the CTA's rows of y are zero
-      if (stack) {
-        for (int i = tid; i < wk.nr * 8 * T; i += kThreads) {
-          const int lr = i / (8 * T), rp = (i / T) % 8, tt = i % T;
-          st_relaxed_u64(ty_l + (static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + 2 * rp) / 2, ytag);
-        }
-      } else {
-        for (int i = tid; i < wk.nr * 16 * T; i += kThreads) {
-          const int lr = i / (16 * T), row = (i / T) % 16, tt = i % T;
-          const size_t yi = static_cast<size_t>(tt) * H + 16 * (wk.r0 + lr) + row;
-          if (a.y32) a.y32[yi] = 0.f;
-          else y_l[yi] = 0;
-        }
+      // expert): CTA c writes zero rows for the tiles split_at(R, c) ..
+      const int R = H / 16, t0r = split_at(R, cta, G), t1r = split_at(R, cta + 1, G);
+      for (int i = tid; i < (t1r - t0r) * 16 * T; i += kThreads) {
+        const int rr = t0r + i / (16 * T), row = (i / T) % 16, tt = i % T;
+        const size_t yi = static_cast<size_t>(tt) * H + 16 * rr + row;
+        if (a.y32) a.y32[yi] = 0.f;
+        else a.y[yi] = 0;
       }
+    }
+    ok = __syncthreads_and(ok && !s_abort);
+    if (stack && tid == 0 && nfin > 0) {  // this CTA's tiles of y are written: count them in
+      __threadfence();
+      red_release_add_u32(a.sync + kSyncY, static_cast<unsigned>(nfin));
     }
     ebase += wk.cnt;
-    MOE_TRACE_POINT(3, 11);
-    // ---- every slot is free: the next layer's first entries (shared-expert
-    // tiles) stream in
-    __syncthreads();
-    lw = lw_next;
-    if (l + 1 < L && ok && predict && warp < npre && lane == 0)
-      issue_entry(a, rg, lw_next, s_pre_expert, pw, warp, ebase + warp);
-  }
-
-  // ---- the stack's final residual and normalised x (CTA 0)
-  if (kStack && ok && cta == 0) {
-    if (residual_norm(a, rs, a.ty + static_cast<size_t>((L - 1) & 1) * T * H / 2, tag0 + (L - 1), xb, red_d, den_s,
-                      &s_abort)) {
-      for (int u = tid; u < T * H / 8; u += kThreads) {
-        reinterpret_cast<uint4*>(a.r_io)[u] = reinterpret_cast<const uint4*>(rs)[u];
-        reinterpret_cast<uint4*>(a.x_io)[u] = reinterpret_cast<const uint4*>(xb)[u];
-      }
+    gbase += wk.ng;
+    MOE_TRACE_LAYER(3, 11);
+    // ---- the next layer's weights (its entries are requested after its
+    // routing: copies requested now would slow the polls of its exchanges)
+    if (tid == 0) {
+      s_lay = s_lay_next;
+      ictx.w13 = s_lay.w13;
+      ictx.w2 = s_lay.w2;
     }
+    __syncthreads();
+    npre = 0;
   }
 
+#undef MOE_TRACE_LAYER
+  MOE_TR(if (lane == 0 && cta < 148) for (int i = 0; i < 8; ++i) g_wcyc[cta][warp][i] = cyc[i];)
   // ---- copies still in flight land before the CTA exits (after a failed
   // wait some may not have been consumed; the last use of every slot is
   // waited for, which returns at once when it completed)
@@ -1104,6 +1278,7 @@ decode_kernel(DecodeArgs a) {
     for (int i = tid; i < L * kMaxDistinct * kMaxTokGemv; i += kThreads) a.amax[i] = 0u;
     if (tid == 0) {
       a.sync[kSyncGU] = 0u;
+      a.sync[kSyncY] = 0u;
       a.sync[kSyncExit] = 0u;
       a.sync[kSyncEpoch] += 1u;  // the next launch's tags differ from every tag of this one
     }
@@ -1118,6 +1293,9 @@ extern "C" int moe_trace_read_decode(unsigned long long* out) {
 }
 extern "C" int moe_trace_read_decode_warps(unsigned long long* out) {
   return cudaMemcpyFromSymbol(out, g_wtrace, sizeof(g_wtrace)) == cudaSuccess ? 0 : -1;
+}
+extern "C" int moe_trace_read_decode_cycles(long long* out) {
+  return cudaMemcpyFromSymbol(out, g_wcyc, sizeof(g_wcyc)) == cudaSuccess ? 0 : -1;
 }
 #endif
 
@@ -1145,6 +1323,7 @@ bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   const int H = a.H, I = a.I, T = a.T;
   if (T < 1 || T > kMaxTokGemv || n_ctas < 1 || a.L < 1) return false;
   if (a.ep_lo < 0 || a.ep_hi > a.E || a.ep_lo >= a.ep_hi) return false;  // the routed experts this call runs
+  if (I / 32 > kDnPB * kWarps) return false;  // a warp's K part of a down slab holds at most kDnPB blocks
   const int R = H / 16;
   const size_t gb = gu_entry_bytes(H), db = dn_entry_bytes(I);
   const size_t slot = up128(gb > db ? gb : db);
@@ -1157,18 +1336,19 @@ bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   // layer start: bf16 x, router partial sums
   a.lpart_off = static_cast<int>(up128(static_cast<size_t>(T) * H * 2));
   const size_t u_start = a.lpart_off + up128(static_cast<size_t>(rr_max) * T * 4 * 8);
-  // down: FP8 h of every pair, the float64 sums of the CTA's row tiles per K part
-  const int nrt = R / n_ctas + 1;
-  a.yrow_len = nrt * ((I / 32 + kPartBlocks - 1) / kPartBlocks) * 16 * T;
+  // down: FP8 h of every pair, the float64 sums per row tile touched and warp
+  const int ntl_max = (R + n_ctas - 1) / n_ctas + 2;
+  a.ypk = (n_ctas + R - 1) / R + 2;
+  a.yrow_len = ntl_max * kWarps * 16 * T;
   a.yrow_off = static_cast<int>(up128(static_cast<size_t>(T) * (a.k + a.n_shared) * I));
   const size_t u_down = a.yrow_off + up128(static_cast<size_t>(a.yrow_len) * 8);
   // the most entries one CTA can have in a layer (slots beyond it are unused)
   const size_t max_d = static_cast<size_t>(T) * a.k + a.n_shared;
-  const size_t bytes = max_d * (I / kFeat) * gb + static_cast<size_t>(R) * max_d * db;
-  const int ent_max = static_cast<int>((bytes / n_ctas + gb - 1) / gb + 2 + (nrt * max_d + a.dpe - 1) / a.dpe);
+  const size_t ent_max = (max_d * (I / kFeat) + n_ctas - 1) / n_ctas +
+                         ((max_d * R + n_ctas - 1) / n_ctas + a.dpe - 1) / a.dpe;
   for (int ns = kMaxNS; ns >= 2; --ns) {
-    if (ns > ent_max && ns > 2) continue;
-    const size_t u_gu = up128(static_cast<size_t>(ns) * kQuarters * 16 * T * 4);
+    if (static_cast<size_t>(ns) > ent_max && ns > 2) continue;
+    const size_t u_gu = up128(static_cast<size_t>(2 * ns) * kWarps * 16 * T * 4);
     size_t u = u_start > u_down ? u_start : u_down;
     if (u_gu > u) u = u_gu;
     size_t off = static_cast<size_t>(ns) * slot;
@@ -1188,6 +1368,12 @@ bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget) {
   }
   return false;
 }
+
+size_t decode_ypart_bytes(int H, int n_ctas) {
+  const int R = H / 16;
+  return static_cast<size_t>(2) * R * ((n_ctas + R - 1) / R + 2) * kMaxTokGemv * 16 * 2 * 8;
+}
+size_t decode_ty_bytes(int H) { return static_cast<size_t>(2) * kMaxTokGemv * (H / 2) * 8; }
 
 namespace {
 

@@ -49,6 +49,7 @@ cudaError_t launch_route_norms(const uint16_t* Wr, int E, int H, float* wnorm, c
 constexpr int kSyncExit = 1;    // CTAs finished
 constexpr int kSyncGU = 2;      // CTAs whose gate/up tiles are finished
 constexpr int kSyncEpoch = 4;   // launches completed (tags of the logits exchange)
+constexpr int kSyncY = 6;       // row tiles of y finished so far (stacked layers)
 constexpr int kSyncWords = 64;
 constexpr int kMaxStackLayers = 128;
 struct LayerW {                 // one layer's weights (device pointers)
@@ -78,7 +79,14 @@ struct DecodeArgs {
   float* h;             // [kMaxDistinct][kMaxTokGemv][I]
   unsigned* amax;       // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;       // [kSyncWords]
-  unsigned long long* ty;  // [2][T][H/2] y of stacked layers: two bf16 | tag << 32 (zero before the first call)
+  // [2][H/16][ypk][T][16][2] float64 partial sums of y of the row tiles
+  // shared by several CTAs, per tile and contributing CTA: the two 32-bit
+  // halves of the value, each | tag << 32 (zero before the first call); ypk
+  // = most CTAs one row tile can have contributions from (decode_plan)
+  unsigned long long* ypart;
+  int ypk;
+  // [2][T][H/2] y of stacked layers: two bf16 | tag << 32 (zero before the first call)
+  unsigned long long* ty;
   int* err;
   moe_debug dbg;        // plain layer only
   uint16_t* dbg_x;      // [L][T][H] input x of every layer, or null
@@ -90,6 +98,10 @@ struct DecodeArgs {
   int rr_off, xq_off, rs_off, u_off, lpart_off, yrow_off, yrow_len, smem_bytes;
 };
 bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget);
+// Bytes of DecodeArgs::ypart for hidden size H, up to MOE_GEMV_MAX_TOKENS
+// tokens and n_ctas CTAs (the SM count), and of DecodeArgs::ty.
+size_t decode_ypart_bytes(int H, int n_ctas);
+size_t decode_ty_bytes(int H);
 cudaError_t launch_decode(const DecodeArgs& a, int n_ctas, cudaStream_t stream);
 int decode_static_smem();
 

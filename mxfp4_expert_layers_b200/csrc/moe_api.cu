@@ -29,6 +29,8 @@ struct moe_handle_s {
   unsigned* sync;      // [kSyncWords]
   unsigned long long* tlogits;  // [kMaxTokGemv][E] tagged logits of the fused decode kernel
   float* wnorm;        // [E + 1] router row norms (many-token router), or null
+  unsigned long long* ypart;  // partial sums of y of the fused decode kernel (DecodeArgs::ypart)
+  size_t ypart_bytes;
   int n_sms;
   int smem_budget;     // dynamic shared memory available to the decode kernel
   moe::PrefillArgs pf; // workspace views of the many-token path (max_tokens > 4)
@@ -123,7 +125,6 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   size_t n_pf = 0;
   if (many)
     for (size_t v : pf_sizes) n_pf += v;
-  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tlog + n_wnorm + n_pf;
   int dev = 0, optin = 0;
   const int static_smem = moe::decode_static_smem();
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -133,6 +134,9 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     delete h;
     return MOE_ERR_CUDA;
   }
+  h->ypart_bytes = moe::decode_ypart_bytes(cfg->hidden, h->n_sms);
+  const size_t n_ypart = up256(h->ypart_bytes);
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tlog + n_wnorm + n_ypart + n_pf;
   h->smem_budget = optin - static_smem - 256;
   if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
     delete h;
@@ -154,6 +158,7 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
   h->tlogits = reinterpret_cast<unsigned long long*>(p); p += n_tlog;
   h->wnorm = n_wnorm ? reinterpret_cast<float*>(p) : nullptr; p += n_wnorm;
+  h->ypart = reinterpret_cast<unsigned long long*>(p); p += n_ypart;
   h->pf = moe::PrefillArgs{};
   if (many) {
     moe::PrefillArgs& f = h->pf;
@@ -241,6 +246,7 @@ int decode_call(moe_handle h, const uint16_t* x, int T, int route, int32_t* ids,
   a.x = x;
   a.ids = ids; a.w = w; a.counts = counts;
   a.tlogits = h->tlogits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.err = h->err;
+  a.ypart = h->ypart;
   a.y = y;
   if (dbg) a.dbg = *dbg;
   if (!moe::decode_plan(a, h->n_sms, h->smem_budget)) return MOE_ERR_UNSUPPORTED;
@@ -342,6 +348,7 @@ int moe_device_error(moe_handle h, cudaStream_t stream) {
         cudaMemset(h->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
         // the launch counter restarts at zero: no tagged logit of an earlier launch may match again
         cudaMemset(h->tlogits, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.n_experts * 8) != cudaSuccess ||
+        cudaMemset(h->ypart, 0, h->ypart_bytes) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }
@@ -456,7 +463,9 @@ struct moe_stack_s {
   float* h;
   unsigned* amax;        // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;
-  unsigned long long* ty;  // [2][kMaxTokGemv][H/2] tagged y of the stacked layers
+  unsigned long long* ypart;  // partial sums of y of the stacked layers (DecodeArgs::ypart)
+  size_t ypart_bytes;
+  unsigned long long* ty;     // y of the stacked layers (DecodeArgs::ty)
   int* err;
   int n_sms;
   int smem_budget;
@@ -490,7 +499,8 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * c.inter * 4);
   const size_t n_amax = up256(static_cast<size_t>(n_layers) * moe::kMaxDistinct * moe::kMaxTokGemv * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
-  const size_t n_ybuf = up256(static_cast<size_t>(2) * moe::kMaxTokGemv * (c.hidden / 2) * 8);
+  s->ypart_bytes = moe::decode_ypart_bytes(c.hidden, s->n_sms);
+  const size_t n_ybuf = up256(s->ypart_bytes) + up256(moe::decode_ty_bytes(c.hidden));
   const size_t n_err = 256;
   const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_ybuf + n_err;
   if (cudaMalloc(&s->ws, bytes) != cudaSuccess) {
@@ -503,7 +513,9 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   s->h = reinterpret_cast<float*>(p); p += n_h;
   s->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
   s->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
-  s->ty = reinterpret_cast<unsigned long long*>(p); p += n_ybuf;
+  s->ypart = reinterpret_cast<unsigned long long*>(p);
+  s->ty = reinterpret_cast<unsigned long long*>(p + up256(s->ypart_bytes));
+  p += n_ybuf;
   s->err = reinterpret_cast<int*>(p);
   moe::LayerW* host = new (std::nothrow) moe::LayerW[n_layers];
   if (!host) {
@@ -545,7 +557,7 @@ int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, in
   a.x = x; a.r_io = r; a.x_io = x; a.eps = eps;
   a.ids = topk_ids; a.w = topk_w;
   a.tlogits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync;
-  a.ty = s->ty; a.err = s->err;
+  a.ypart = s->ypart; a.ty = s->ty; a.err = s->err;
   a.dbg_x = x_layers;
   if (!moe::decode_plan(a, s->n_sms, s->smem_budget)) return MOE_ERR_UNSUPPORTED;
   if (s->profiling) s->prof.before(1, stream);
@@ -564,7 +576,8 @@ int moe_stack_device_error(moe_stack s, cudaStream_t stream) {
         cudaMemset(s->amax, 0, static_cast<size_t>(s->L) * moe::kMaxDistinct * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(s->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
         cudaMemset(s->logits, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.n_experts * 8) != cudaSuccess ||
-        cudaMemset(s->ty, 0, static_cast<size_t>(2) * moe::kMaxTokGemv * (s->cfg.hidden / 2) * 8) != cudaSuccess ||
+        cudaMemset(s->ypart, 0, s->ypart_bytes) != cudaSuccess ||
+        cudaMemset(s->ty, 0, moe::decode_ty_bytes(s->cfg.hidden)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }
