@@ -29,6 +29,13 @@ static __device__ unsigned long long g_trace[4][512][64];
       g_trace[k][blockIdx.x + gridDim.x * blockIdx.y][slot] = t_;                   \
     }                                                                               \
   } while (0)
+// The same from whichever thread executes it.
+#define MOE_TRACE_HERE(k, slot)                                                     \
+  do {                                                                              \
+    unsigned long long t_;                                                          \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                          \
+    g_trace[k][blockIdx.x + gridDim.x * blockIdx.y][slot] = t_;                     \
+  } while (0)
 // Per-warp timestamps (lane 0 of each warp of the first 148 CTAs).
 static __device__ unsigned long long g_wtrace[148][16][16];
 #define MOE_WTRACE(slot)                                                            \
@@ -46,6 +53,9 @@ static __device__ long long g_wcyc[148][16][8];
 #define MOE_TR(...) __VA_ARGS__
 #else
 #define MOE_TR(...)
+#define MOE_TRACE_HERE(k, slot) \
+  do {                          \
+  } while (0)
 #define MOE_TRACE_POINT(k, slot) \
   do {                           \
   } while (0)

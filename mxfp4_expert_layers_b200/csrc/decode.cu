@@ -551,7 +551,6 @@ decode_kernel(DecodeArgs a) {
   __shared__ __align__(8) uint64_t full[kMaxNS];
   __shared__ __align__(8) uint64_t fr;
   __shared__ int iss[kMaxNS], arr[kMaxNS];
-  __shared__ int parr[2 * kMaxNS];  // part sums written into each gate/up partial area so far
   __shared__ int freed[kMaxNS];     // entries of each slot consumed so far
   __shared__ int s_riss;  // router-row copies issued
   __shared__ Distinct dist;
@@ -624,7 +623,6 @@ decode_kernel(DecodeArgs a) {
   // ---- before the dependency wait: the first layer's router rows and
   // shared-expert tiles (weights only)
   if (tid < kMaxNS) { iss[tid] = 0; arr[tid] = 0; }
-  if (tid < 2 * kMaxNS) parr[tid] = 0;
   if (tid < kMaxNS) freed[tid] = 0;
   if (tid == 0) {
     for (int s = 0; s < a.ns; ++s) mbar_init(&full[s], 1);
@@ -769,7 +767,19 @@ decode_kernel(DecodeArgs a) {
         st_relaxed_u64(a.tlogits + static_cast<size_t>(tt) * E + row0 + ri,
                        static_cast<unsigned long long>(tag) << 32 | __float_as_uint(lg));
       }
-      __syncthreads();
+      // the hand-off: every CTA counts itself in once its logits are written;
+      // the words are read once the count is complete (polling the words
+      // themselves costs the CTAs that start polling first)
+      if (tid == 0 && ok) {
+        __threadfence();
+        red_release_add_u32(a.sync + kSyncRoute, 1u);
+        if (!poll_geq_bounded(a.sync + kSyncRoute, static_cast<unsigned>((l + 1) * G), a.err)) {
+          ok = false;
+          note_timeout(__LINE__, l, -1);
+        }
+      }
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
       MOE_TRACE_LAYER(3, 3);
       if (warp < T && ok &&
           !topk_warp(a.tlogits + static_cast<size_t>(warp) * E, tag, E, a.k, s_ids + warp * a.k, s_w + warp * a.k,
@@ -810,12 +820,6 @@ decode_kernel(DecodeArgs a) {
       ok = false;
       break;
     }
-    // gate/up tiles first; the down slabs that also fit in the ring follow as
-    // soon as the CTA's first routed tile has landed (so they do not compete
-    // with the gate/up bytes, which the critical path waits for; the down
-    // bytes are needed only after the gate/up barrier)
-    const int first_routed = wk.ng > 0 && wk.g0 + wk.ng > S * cpe ? max(0, S * cpe - wk.g0) : -1;
-    const int dn_lo = max(wk.ng, npre), dn_hi = min(wk.cnt, rg.ns);
     // pair table of the down step (off the critical path): the (expert,
     // token) pairs in order, numbered by a ballot prefix count
     if (warp == kWarps - 1) {
@@ -839,101 +843,101 @@ decode_kernel(DecodeArgs a) {
     // ---- 3. gate/up + SwiGLU: warp w takes the K part w of every tile
     // (blocks w nb / W .. (w + 1) nb / W, W warps), so all warps work on the tile
     // that landed first
-    if (warp == kProducer) {
-      // the producer: the layer's first entries, then each entry whose slot
-      // held a gate/up tile as soon as that tile is consumed
-      if (lane == 0) {
-        bool pok = true;
-        for (int j = npre; j < min(wk.ng, rg.ns); ++j) issue_entry(&ictx, dist.expert, &s_wk, j, ebase + j);
-        if (dn_lo < dn_hi) {
-          if (first_routed >= 0) pok = wait_entry(rg, ebase + first_routed, a.err, &s_abort);
-          for (int j = dn_lo; j < dn_hi && pok; ++j) issue_entry(&ictx, dist.expert, &s_wk, j, ebase + j);
-        }
-        for (int n = rg.ns; n < wk.cnt && n - rg.ns < wk.ng && pok; ++n) {
-          const int gi = ebase + n;
-          pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
-          if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
-        }
-      }
-      __syncwarp();
-    } else {
+    {
       const int g = lane >> 2, t4 = lane & 3;
-      const int b0 = warp * nb / kWarps, b1 = (warp + 1) * nb / kWarps;
       unsigned* amax_l = a.amax + static_cast<size_t>(l) * kMaxDistinct * kMaxTokGemv;
-      const int pslot = kWarps * 16 * T;  // partial sums per slot
-      for (int j = 0; j < wk.ng; ++j) {
-        const int gidx = ebase + j, s = gidx % rg.ns;
-        MOE_TR(long long c0 = clock64();)
-        if (!wait_entry(rg, gidx, a.err, &s_abort)) {
-          if (lane == 0) note_timeout(__LINE__, l, gidx);
-          break;
-        }
-        MOE_TR(cyc[4] += clock64() - c0;)
-        if (j < 8 && warp == 0) MOE_TRACE_LAYER(3, 20 + j);
-        MOE_WTRACE(min(j, 3) * 2);
-        const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot;
-        const int i = wk.g0 + j, u = i / cpe, f0 = (i % cpe) * kFeat;
-        const bool tok = g < T && (dist.mask[u] >> g & 1);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        MOE_TR(c0 = clock64();)
-        tile_blocks<kTc>(st, nb, b0, b1, tok ? xq + static_cast<size_t>(g) * H + 8 * t4 : nullptr, acc);
-        MOE_TR(cyc[0] += clock64() - c0; cyc[1] += 1;)
-        MOE_WTRACE(min(j, 3) * 2 + 1);
-        // this warp's part sums go to partial area pa, by the launch-wide
-        // gate/up tile number gt (2 ns areas: a warp may start on tile gt + ns
-        // before the epilogue of tile gt has read them, but not on gt + 2 ns,
-        // whose weights need a slot that the epilogue's warp frees after it)
-        const int gt = gbase + j, pa = gt % (2 * rg.ns), puse = gt / (2 * rg.ns);
-        float* red = redp + static_cast<size_t>(pa) * pslot + warp * 16 * T;
-        if (2 * t4 < T) {
-          red[g * T + 2 * t4] = acc[0];
-          red[(g + 8) * T + 2 * t4] = acc[2];
-          if (!kT1 && 2 * t4 + 1 < T) {
-            red[g * T + 2 * t4 + 1] = acc[1];
-            red[(g + 8) * T + 2 * t4 + 1] = acc[3];
+      const int pslot = kWarps * 16 * T;  // part sums per partial area
+      if (warp == kProducer) {
+        // the producer requests every weight copy (a request waits while
+        // the copy engine is busy, so no other warp makes one): the layer's
+        // first entries at once, then each entry as soon as the previous
+        // entry of its slot has been consumed
+        if (lane == 0) {
+          bool pok = true;
+          for (int n = npre; n < min(wk.cnt, rg.ns); ++n) issue_entry(&ictx, dist.expert, &s_wk, n, ebase + n);
+          for (int n = rg.ns; n < wk.cnt && n - rg.ns < wk.ng && pok; ++n) {
+            const int gi = ebase + n;
+            pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
+            if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
           }
+          MOE_TR(if (l == L - 1) MOE_TRACE_HERE(3, 14);)
         }
         __syncwarp();
-        if (lane == 0) {
-          __threadfence_block();
-          atomicAdd(&parr[pa], 1);
-          // the last warp done with the slot's weights frees it (the producer
-          // requests its next entry)
-          if (atomicAdd(&rg.arr[s], 1) == kWarps - 1) {
-            rg.arr[s] = 0;
+      } else {
+        // compute warp w: the K part w of every tile (blocks w nb / W ..
+        // (w + 1) nb / W, W compute warps), tiles in order; the last warp to
+        // finish a tile frees its slot and runs its epilogue
+        const int b0 = warp * nb / kWarps, b1 = (warp + 1) * nb / kWarps;
+        for (int j = 0; j < wk.ng; ++j) {
+          const int gidx = ebase + j, s = gidx % rg.ns;
+          MOE_TR(long long c0 = clock64();)
+          if (!wait_entry(rg, gidx, a.err, &s_abort)) {
+            if (lane == 0) note_timeout(__LINE__, l, gidx);
+            break;
+          }
+          MOE_TR(cyc[4] += clock64() - c0;)
+          if (j < 8 && warp == 0) MOE_TRACE_LAYER(3, 20 + j);
+          MOE_WTRACE(min(j, 3) * 2);
+          const uint8_t* st = rg.base + static_cast<size_t>(s) * rg.slot;
+          const int i = wk.g0 + j, u = i / cpe, f0 = (i % cpe) * kFeat;
+          const bool tok = g < T && (dist.mask[u] >> g & 1);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          MOE_TR(c0 = clock64();)
+          tile_blocks<kTc>(st, nb, b0, b1, tok ? xq + static_cast<size_t>(g) * H + 8 * t4 : nullptr, acc);
+          MOE_TR(cyc[0] += clock64() - c0; cyc[1] += 1;)
+          MOE_WTRACE(min(j, 3) * 2 + 1);
+          // part sums to partial area pa, by the launch-wide gate/up tile
+          // number gt (2 ns areas, so that the sums of tile gt + ns cannot
+          // overwrite those of tile gt before its epilogue has read them)
+          const int gt = gbase + j, pa = gt % (2 * rg.ns);
+          float* red = redp + static_cast<size_t>(pa) * pslot + warp * 16 * T;
+          if (2 * t4 < T) {
+            red[g * T + 2 * t4] = acc[0];
+            red[(g + 8) * T + 2 * t4] = acc[2];
+            if (!kT1 && 2 * t4 + 1 < T) {
+              red[g * T + 2 * t4 + 1] = acc[1];
+              red[(g + 8) * T + 2 * t4 + 1] = acc[3];
+            }
+          }
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) {
             __threadfence_block();
-            atomicAdd(&freed[s], 1);
+            last = atomicAdd(&rg.arr[s], 1) == kWarps - 1;
+            if (last) {
+              rg.arr[s] = 0;
+              atomicAdd(&freed[s], 1);  // the producer may refill the slot
+            }
+            __threadfence_block();
           }
-        }
-        // the epilogue of tile j: warp j mod W, once every warp's part sums
-        // are in (a rotating warp, so that no warp does it for every tile)
-        if (warp != j % kWarps) continue;
-        if (lane == 0 && !wait_count(&parr[pa], kWarps * (puse + 1), a.err, &s_abort)) note_timeout(__LINE__, l, gidx);
-        __syncwarp();  // lane 0's acquire orders the other lanes' reads too
-        if (j < 8) MOE_TRACE_LAYER(3, 28 + j);
-        // the parts' sums of feature f, token tt (lanes o = f * T + tt), in part order
-        const float* rs4 = redp + static_cast<size_t>(pa) * pslot;
-        double gs = 0.0, us = 0.0;
-        const int f = lane / T, tt = lane % T;
-        if (lane < kFeat * T) {
-#pragma unroll 4
-          for (int q = 0; q < kWarps; ++q) {
-            gs += rs4[(q * 16 + f) * T + tt];
-            us += rs4[(q * 16 + f + 8) * T + tt];
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (!last) continue;
+          __syncwarp();  // lane 0's acquire orders the other lanes' reads too
+          if (j < 8) MOE_TRACE_LAYER(3, 28 + j);
+          // the parts' sums of feature f, token tt (lanes o = f * T + tt), in part order
+          const float* rs4 = redp + static_cast<size_t>(pa) * pslot;
+          double gs = 0.0, us = 0.0;
+          const int f = lane / T, tt = lane % T;
+          if (lane < kFeat * T) {
+#pragma unroll
+            for (int q = 0; q < kWarps; ++q) {
+              gs += rs4[(q * 16 + f) * T + tt];
+              us += rs4[(q * 16 + f + 8) * T + tt];
+            }
           }
+          if (lane < kFeat * T && (dist.mask[u] >> tt & 1)) {
+            const float gv = static_cast<float>(static_cast<double>(xs[tt]) * gs);
+            const float uv = static_cast<float>(static_cast<double>(xs[tt]) * us);
+            const float hv = gv / (1.0f + expf(-gv)) * uv;  // SwiGLU (float32)
+            __stcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + f0 + f, hv);
+            const float m = fabsf(hv);
+            if (m > 0.f) red_max_u32(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
+          }
+          if (j < 8) MOE_TRACE_LAYER(3, 40 + j);
         }
-        if (lane < kFeat * T && (dist.mask[u] >> tt & 1)) {
-          // SwiGLU in float32 (a short dependency chain)
-          const float gv = static_cast<float>(static_cast<double>(xs[tt]) * gs);
-          const float uv = static_cast<float>(static_cast<double>(xs[tt]) * us);
-          const float hv = gv / (1.0f + expf(-gv)) * uv;
-          __stcg(a.h + (static_cast<size_t>(u) * kMaxTokGemv + tt) * I + f0 + f, hv);
-          const float m = fabsf(hv);
-          if (m > 0.f) red_max_u32(amax_l + u * kMaxTokGemv + tt, __float_as_uint(m));
-        }
-        if (j < 8) MOE_TRACE_LAYER(3, 40 + j);
       }
     }
+    MOE_WTRACE(7);
     ok = __syncthreads_and(!s_abort);
     if (!ok) break;
     MOE_TRACE_LAYER(3, 7);
@@ -1279,6 +1283,7 @@ decode_kernel(DecodeArgs a) {
     if (tid == 0) {
       a.sync[kSyncGU] = 0u;
       a.sync[kSyncY] = 0u;
+      a.sync[kSyncRoute] = 0u;
       a.sync[kSyncExit] = 0u;
       a.sync[kSyncEpoch] += 1u;  // the next launch's tags differ from every tag of this one
     }

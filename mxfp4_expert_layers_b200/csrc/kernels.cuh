@@ -50,6 +50,7 @@ constexpr int kSyncExit = 1;    // CTAs finished
 constexpr int kSyncGU = 2;      // CTAs whose gate/up tiles are finished
 constexpr int kSyncEpoch = 4;   // launches completed (tags of the logits exchange)
 constexpr int kSyncY = 6;       // row tiles of y finished so far (stacked layers)
+constexpr int kSyncRoute = 7;   // CTAs whose router logits are written, summed over layers
 constexpr int kSyncWords = 64;
 constexpr int kMaxStackLayers = 128;
 struct LayerW {                 // one layer's weights (device pointers)
