@@ -298,28 +298,66 @@ __device__ __forceinline__ int weight_index(const IssueCtx* c, int e) {
   return e < c->E ? e - c->ep_lo : (c->ep_hi - c->ep_lo) + (e - c->E);
 }
 
-// Request entry j of the layer (launch-wide entry gidx) into its slot.
-// `expert` maps distinct-expert positions to expert indices.
+// Request entry j of the layer (launch-wide entry gidx) into its slot; all 32
+// lanes of the producer warp call it, and each copy is requested by its own
+// lane (a copy request keeps its thread about 200 ns; the requests of
+// different lanes overlap).  `expert` maps distinct-expert positions to
+// expert indices.
 __device__ __noinline__ void issue_entry(const IssueCtx* c, const int* expert, const Work* wk, int j, int gidx) {
+  const int lane = threadIdx.x & 31;
   const int s = gidx % c->ns;
   uint8_t* dst = c->ring + static_cast<size_t>(s) * c->slot;
   if (j < wk->ng) {
     const int cpe = c->I / kFeat, i = wk->g0 + j, bytes = gu_entry_bytes(c->H);
-    mbar_expect_tx(&c->full[s], static_cast<uint32_t>(bytes));
-    bulk_g2s(dst, c->w13 + (static_cast<size_t>(weight_index(c, expert[i / cpe])) * cpe + i % cpe) * bytes,
-             static_cast<uint32_t>(bytes), &c->full[s]);
+    if (lane == 0) {
+      mbar_expect_tx(&c->full[s], static_cast<uint32_t>(bytes));
+      bulk_g2s(dst, c->w13 + (static_cast<size_t>(weight_index(c, expert[i / cpe])) * cpe + i % cpe) * bytes,
+               static_cast<uint32_t>(bytes), &c->full[s]);
+    }
   } else {
     const int d = j - wk->ng, ka = d * c->dpe, n = min(c->dpe, wk->nq - ka);
     const int bytes = dn_entry_bytes(c->I), R = c->H / 16;
-    mbar_expect_tx(&c->full[s], static_cast<uint32_t>(n * bytes));
-    for (int k = ka; k < ka + n; ++k) {
-      const int sl = wk->s0 + k;
-      bulk_g2s(dst + (k - ka) * bytes,
+    if (lane == 0) mbar_expect_tx(&c->full[s], static_cast<uint32_t>(n * bytes));
+    __syncwarp();
+    for (int k = lane; k < n; k += 32) {
+      const int sl = wk->s0 + ka + k;
+      bulk_g2s(dst + k * bytes,
                c->w2 + (static_cast<size_t>(weight_index(c, expert[sl % wk->nd])) * R + sl / wk->nd) * bytes,
                static_cast<uint32_t>(bytes), &c->full[s]);
     }
   }
-  atomicAdd(&c->iss[s], 1);
+  __syncwarp();
+  if (lane == 0) atomicAdd(&c->iss[s], 1);
+}
+
+// Request entries j0 .. j1-1 of the layer (launch-wide gidx0 + j - j0), each by
+// one lane of the producer warp (all 32 lanes call it; at most 32 entries),
+// for the first entries of a layer: they go to distinct slots.
+__device__ __noinline__ void issue_entries(const IssueCtx* c, const int* expert, const Work* wk, int j0, int j1,
+                                           int gidx0) {
+  const int lane = threadIdx.x & 31, j = j0 + lane;
+  if (j < j1) {
+    const int gidx = gidx0 + lane, s = gidx % c->ns;
+    uint8_t* dst = c->ring + static_cast<size_t>(s) * c->slot;
+    if (j < wk->ng) {
+      const int cpe = c->I / kFeat, i = wk->g0 + j, bytes = gu_entry_bytes(c->H);
+      mbar_expect_tx(&c->full[s], static_cast<uint32_t>(bytes));
+      bulk_g2s(dst, c->w13 + (static_cast<size_t>(weight_index(c, expert[i / cpe])) * cpe + i % cpe) * bytes,
+               static_cast<uint32_t>(bytes), &c->full[s]);
+    } else {
+      const int d = j - wk->ng, ka = d * c->dpe, n = min(c->dpe, wk->nq - ka);
+      const int bytes = dn_entry_bytes(c->I), R = c->H / 16;
+      mbar_expect_tx(&c->full[s], static_cast<uint32_t>(n * bytes));
+      for (int k = 0; k < n; ++k) {
+        const int sl = wk->s0 + ka + k;
+        bulk_g2s(dst + k * bytes,
+                 c->w2 + (static_cast<size_t>(weight_index(c, expert[sl % wk->nd])) * R + sl / wk->nd) * bytes,
+                 static_cast<uint32_t>(bytes), &c->full[s]);
+      }
+    }
+    atomicAdd(&c->iss[s], 1);
+  }
+  __syncwarp();
 }
 
 // Wait until entry gidx has landed in its slot: first until it has been
@@ -638,13 +676,13 @@ decode_kernel(DecodeArgs a) {
   // (every weight copy is requested by one thread, lane 0 of the producer
   // warp: a copy request waits while the copy engine's queue is full, and
   // that wait must not hold up the warps that compute)
-  if (warp == kProducer && lane == 0) {
-    if (nrr > 0) {
+  if (warp == kProducer) {
+    if (lane == 0 && nrr > 0) {
       mbar_expect_tx(&fr, static_cast<uint32_t>(nrr * H * 2));
       bulk_g2s(rr, s_lay.Wr + static_cast<size_t>(row0) * H, static_cast<uint32_t>(nrr * H * 2), &fr);
       s_riss = 1;
     }
-    for (int j = 0; j < npre; ++j) issue_entry(&ictx, s_pre_expert, &s_pw, j, j);
+    if (npre > 0) issue_entries(&ictx, s_pre_expert, &s_pw, 0, npre, 0);
   }
   int ebase = 0;  // launch-wide number of this layer's entry 0
   int gbase = 0;  // launch-wide number of this layer's gate/up tile 0
@@ -852,16 +890,15 @@ decode_kernel(DecodeArgs a) {
         // the copy engine is busy, so no other warp makes one): the layer's
         // first entries at once, then each entry as soon as the previous
         // entry of its slot has been consumed
-        if (lane == 0) {
-          bool pok = true;
-          for (int n = npre; n < min(wk.cnt, rg.ns); ++n) issue_entry(&ictx, dist.expert, &s_wk, n, ebase + n);
-          for (int n = rg.ns; n < wk.cnt && n - rg.ns < wk.ng && pok; ++n) {
-            const int gi = ebase + n;
-            pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
-            if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
-          }
-          MOE_TR(if (l == L - 1) MOE_TRACE_HERE(3, 14);)
+        if (npre < min(wk.cnt, rg.ns)) issue_entries(&ictx, dist.expert, &s_wk, npre, min(wk.cnt, rg.ns), ebase + npre);
+        for (int n = rg.ns; n < wk.cnt && n - rg.ns < wk.ng; ++n) {
+          const int gi = ebase + n;
+          int pok = 1;
+          if (lane == 0) pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
+          if (!__shfl_sync(0xffffffffu, pok, 0)) break;
+          issue_entry(&ictx, dist.expert, &s_wk, n, gi);
         }
+        MOE_TR(if (l == L - 1 && lane == 0) MOE_TRACE_HERE(3, 14);)
         __syncwarp();
       } else {
         // compute warp w: the K part w of every tile (blocks w nb / W ..
@@ -1083,15 +1120,14 @@ decode_kernel(DecodeArgs a) {
       if (warp == kProducer) {
         // the producer: each entry whose slot held a down entry as soon as
         // that is consumed; then the next layer's router rows
-        if (lane == 0) {
-          bool pok = true;
-          for (int n = max(rg.ns, wk.ng + rg.ns); n < wk.cnt && pok; ++n) {
-            const int gi = ebase + n;
-            pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
-            if (pok) issue_entry(&ictx, dist.expert, &s_wk, n, gi);
-          }
-          prefetch_router();
+        for (int n = max(rg.ns, wk.ng + rg.ns); n < wk.cnt; ++n) {
+          const int gi = ebase + n;
+          int pok = 1;
+          if (lane == 0) pok = wait_count(&freed[gi % rg.ns], gi / rg.ns, a.err, &s_abort);
+          if (!__shfl_sync(0xffffffffu, pok, 0)) break;
+          issue_entry(&ictx, dist.expert, &s_wk, n, gi);
         }
+        if (lane == 0) prefetch_router();
         __syncwarp();
       } else {
       bool good = true;

@@ -100,23 +100,8 @@ __device__ unsigned long long g_tc_trace[2][4][12][64];
   } while (0)
 #endif
 
-// K-major, no swizzle: core matrices of 8 rows x 16 bytes; LBO = next 16-byte
-// piece along K (128 B), SBO = next 8-row band.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-
 // canonical K-major byte offset of row r, byte k of the chunk
 __device__ __forceinline__ int canon(int r, int k) { return (r >> 3) * kSBO + (k >> 4) * 128 + (r & 7) * 16 + (k & 15); }
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
-               : "memory");
-}
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
