@@ -46,11 +46,10 @@ cudaError_t launch_route_norms(const uint16_t* Wr, int E, int H, float* wnorm, c
 // Fused decode pass, T <= MOE_GEMV_MAX_TOKENS (decode.cu): one persistent
 // launch for one layer or a chained stack of layers (routing optional for a
 // single layer; required for a stack).
+constexpr int kSyncRoute = 0;   // grid arrive/wait counter of the routing step
 constexpr int kSyncExit = 1;    // CTAs finished
 constexpr int kSyncGU = 2;      // CTAs whose gate/up tiles are finished
-constexpr int kSyncEpoch = 4;   // launches completed (tags of the logits exchange)
-constexpr int kSyncY = 6;       // row tiles of y finished so far (stacked layers)
-constexpr int kSyncRoute = 7;   // CTAs whose router logits are written, summed over layers
+constexpr int kSyncY = 3;       // CTAs whose part of y is written
 constexpr int kSyncWords = 64;
 constexpr int kMaxStackLayers = 128;
 struct LayerW {                 // one layer's weights (device pointers)
@@ -76,33 +75,21 @@ struct DecodeArgs {
   uint16_t* y;          // [T][H] output of a plain layer
   float* y32;           // [T][H] float32 part of y from this call's experts (replaces y), or null
   // workspace; the counters and accumulators are zero between calls
-  unsigned long long* tlogits;  // [kMaxTokGemv][E] logit bits | tag << 32 (zero before the first call)
+  float* logits;        // [T][E]
   float* h;             // [kMaxDistinct][kMaxTokGemv][I]
   unsigned* amax;       // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;       // [kSyncWords]
-  // [2][H/16][ypk][T][16][2] float64 partial sums of y of the row tiles
-  // shared by several CTAs, per tile and contributing CTA: the two 32-bit
-  // halves of the value, each | tag << 32 (zero before the first call); ypk
-  // = most CTAs one row tile can have contributions from (decode_plan)
-  unsigned long long* ypart;
-  int ypk;
-  // [2][T][H/2] y of stacked layers: two bf16 | tag << 32 (zero before the first call)
-  unsigned long long* ty;
+  unsigned* tile_cnt;   // [H/16]
+  double* yacc;         // [kMaxTokGemv][H]
+  uint16_t* ybuf;       // [2][T][H] y of stacked layers
   int* err;
   moe_debug dbg;        // plain layer only
   uint16_t* dbg_x;      // [L][T][H] input x of every layer, or null
-  // shared-memory plan (decode_plan): the weight ring (ns slots of
-  // slot_bytes, a down entry holds dpe slabs), then the regions at the
-  // given byte offsets; u_off starts the region shared by the layer start,
-  // gate/up and down (lpart_off, yrow_off relative to it)
-  int ns, slot_bytes, dpe;
-  int rr_off, xq_off, rs_off, u_off, lpart_off, yrow_off, yrow_len, smem_bytes;
+  // shared-memory plan (decode_plan)
+  int ng_slots, nd_slots;  // gate/up and down ring slots
+  int dn_off, rr_off, xq_off, red_off, qh_off, yrow_off, rs_off, yrow_len, smem_bytes;
 };
 bool decode_plan(DecodeArgs& a, int n_ctas, int smem_budget);
-// Bytes of DecodeArgs::ypart for hidden size H, up to MOE_GEMV_MAX_TOKENS
-// tokens and n_ctas CTAs (the SM count), and of DecodeArgs::ty.
-size_t decode_ypart_bytes(int H, int n_ctas);
-size_t decode_ty_bytes(int H);
 cudaError_t launch_decode(const DecodeArgs& a, int n_ctas, cudaStream_t stream);
 int decode_static_smem();
 

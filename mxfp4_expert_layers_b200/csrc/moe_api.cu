@@ -27,10 +27,9 @@ struct moe_handle_s {
   unsigned* amax;      // [kMaxDistinct][kMaxTokGemv]
   float* h;            // [kMaxDistinct][kMaxTokGemv][I]
   unsigned* sync;      // [kSyncWords]
-  unsigned long long* tlogits;  // [kMaxTokGemv][E] tagged logits of the fused decode kernel
+  unsigned* tile_cnt;  // [H/16] contributions counted in per shared row tile (fused decode kernel)
+  double* yacc;        // [kMaxTokGemv][H] float64 sums of shared row tiles (fused decode kernel)
   float* wnorm;        // [E + 1] router row norms (many-token router), or null
-  unsigned long long* ypart;  // partial sums of y of the fused decode kernel (DecodeArgs::ypart)
-  size_t ypart_bytes;
   int n_sms;
   int smem_budget;     // dynamic shared memory available to the decode kernel
   moe::PrefillArgs pf; // workspace views of the many-token path (max_tokens > 4)
@@ -98,7 +97,8 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   const size_t n_amax = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * I * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
-  const size_t n_tlog = up256(static_cast<size_t>(moe::kMaxTokGemv) * E * 8);
+  const size_t n_tcnt = up256(static_cast<size_t>(cfg->hidden / 16) * 4);
+  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * cfg->hidden * 8);
   const size_t n_wnorm = max_tokens > moe::kRouteGemmMinTokens ? up256(static_cast<size_t>(E + 1) * 4) : 0;
   // the many-token path: pairs P = max_tokens * (k + S)
   const size_t T = static_cast<size_t>(max_tokens), H = cfg->hidden, NE = E + cfg->n_shared;
@@ -134,9 +134,7 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
     delete h;
     return MOE_ERR_CUDA;
   }
-  h->ypart_bytes = moe::decode_ypart_bytes(cfg->hidden, h->n_sms);
-  const size_t n_ypart = up256(h->ypart_bytes);
-  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tlog + n_wnorm + n_ypart + n_pf;
+  h->ws_bytes = n_logits + n_tiles + n_small + n_amax + n_h + n_sync + n_tcnt + n_yacc + n_wnorm + n_pf;
   h->smem_budget = optin - static_smem - 256;
   if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
     delete h;
@@ -156,9 +154,9 @@ int moe_create(const moe_config* cfg, const moe_weights* weights, int max_tokens
   h->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
   h->h = reinterpret_cast<float*>(p); p += n_h;
   h->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
-  h->tlogits = reinterpret_cast<unsigned long long*>(p); p += n_tlog;
+  h->tile_cnt = reinterpret_cast<unsigned*>(p); p += n_tcnt;
+  h->yacc = reinterpret_cast<double*>(p); p += n_yacc;
   h->wnorm = n_wnorm ? reinterpret_cast<float*>(p) : nullptr; p += n_wnorm;
-  h->ypart = reinterpret_cast<unsigned long long*>(p); p += n_ypart;
   h->pf = moe::PrefillArgs{};
   if (many) {
     moe::PrefillArgs& f = h->pf;
@@ -245,8 +243,8 @@ int decode_call(moe_handle h, const uint16_t* x, int T, int route, int32_t* ids,
   a.layer0 = moe::LayerW{h->w.router_w, h->w.router_bias, h->w.w13, h->w.w2};
   a.x = x;
   a.ids = ids; a.w = w; a.counts = counts;
-  a.tlogits = h->tlogits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.err = h->err;
-  a.ypart = h->ypart;
+  a.logits = h->logits; a.h = h->h; a.amax = h->amax; a.sync = h->sync; a.tile_cnt = h->tile_cnt;
+  a.yacc = h->yacc; a.err = h->err;
   a.y = y;
   if (dbg) a.dbg = *dbg;
   if (!moe::decode_plan(a, h->n_sms, h->smem_budget)) return MOE_ERR_UNSUPPORTED;
@@ -346,9 +344,8 @@ int moe_device_error(moe_handle h, cudaStream_t stream) {
     if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
         cudaMemset(h->amax, 0, static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(h->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
-        // the launch counter restarts at zero: no tagged logit of an earlier launch may match again
-        cudaMemset(h->tlogits, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.n_experts * 8) != cudaSuccess ||
-        cudaMemset(h->ypart, 0, h->ypart_bytes) != cudaSuccess ||
+        cudaMemset(h->tile_cnt, 0, static_cast<size_t>(h->cfg.hidden / 16) * 4) != cudaSuccess ||
+        cudaMemset(h->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * h->cfg.hidden * 8) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }
@@ -459,13 +456,13 @@ struct moe_stack_s {
   int max_tokens;
   void* ws;
   moe::LayerW* layers;   // [L] device
-  unsigned long long* logits;  // [kMaxTokGemv][E] tagged logits
+  float* logits;         // [kMaxTokGemv][E]
   float* h;
   unsigned* amax;        // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;
-  unsigned long long* ypart;  // partial sums of y of the stacked layers (DecodeArgs::ypart)
-  size_t ypart_bytes;
-  unsigned long long* ty;     // y of the stacked layers (DecodeArgs::ty)
+  unsigned* tile_cnt;
+  double* yacc;
+  uint16_t* ybuf;        // [2][kMaxTokGemv][H] y of the stacked layers
   int* err;
   int n_sms;
   int smem_budget;
@@ -495,12 +492,13 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   s->n_sms = layers[0]->n_sms;
   s->smem_budget = layers[0]->smem_budget;
   const size_t n_layers_b = up256(static_cast<size_t>(n_layers) * sizeof(moe::LayerW));
-  const size_t n_logits = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.n_experts * 8);
+  const size_t n_logits = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.n_experts * 4);
   const size_t n_h = up256(static_cast<size_t>(moe::kMaxDistinct) * moe::kMaxTokGemv * c.inter * 4);
   const size_t n_amax = up256(static_cast<size_t>(n_layers) * moe::kMaxDistinct * moe::kMaxTokGemv * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
-  s->ypart_bytes = moe::decode_ypart_bytes(c.hidden, s->n_sms);
-  const size_t n_ybuf = up256(s->ypart_bytes) + up256(moe::decode_ty_bytes(c.hidden));
+  const size_t n_tcnt = up256(static_cast<size_t>(c.hidden / 16) * 4);
+  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.hidden * 8);
+  const size_t n_ybuf = n_tcnt + n_yacc + up256(static_cast<size_t>(2) * moe::kMaxTokGemv * c.hidden * 2);
   const size_t n_err = 256;
   const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_ybuf + n_err;
   if (cudaMalloc(&s->ws, bytes) != cudaSuccess) {
@@ -509,12 +507,13 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   }
   uint8_t* p = static_cast<uint8_t*>(s->ws);
   s->layers = reinterpret_cast<moe::LayerW*>(p); p += n_layers_b;
-  s->logits = reinterpret_cast<unsigned long long*>(p); p += n_logits;
+  s->logits = reinterpret_cast<float*>(p); p += n_logits;
   s->h = reinterpret_cast<float*>(p); p += n_h;
   s->amax = reinterpret_cast<unsigned*>(p); p += n_amax;
   s->sync = reinterpret_cast<unsigned*>(p); p += n_sync;
-  s->ypart = reinterpret_cast<unsigned long long*>(p);
-  s->ty = reinterpret_cast<unsigned long long*>(p + up256(s->ypart_bytes));
+  s->tile_cnt = reinterpret_cast<unsigned*>(p);
+  s->yacc = reinterpret_cast<double*>(p + n_tcnt);
+  s->ybuf = reinterpret_cast<uint16_t*>(p + n_tcnt + n_yacc);
   p += n_ybuf;
   s->err = reinterpret_cast<int*>(p);
   moe::LayerW* host = new (std::nothrow) moe::LayerW[n_layers];
@@ -556,8 +555,8 @@ int moe_stack_decode(moe_stack s, uint16_t* r, uint16_t* x, int T, float eps, in
   a.layers = s->layers;
   a.x = x; a.r_io = r; a.x_io = x; a.eps = eps;
   a.ids = topk_ids; a.w = topk_w;
-  a.tlogits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync;
-  a.ypart = s->ypart; a.ty = s->ty; a.err = s->err;
+  a.logits = s->logits; a.h = s->h; a.amax = s->amax; a.sync = s->sync; a.tile_cnt = s->tile_cnt;
+  a.yacc = s->yacc; a.ybuf = s->ybuf; a.err = s->err;
   a.dbg_x = x_layers;
   if (!moe::decode_plan(a, s->n_sms, s->smem_budget)) return MOE_ERR_UNSUPPORTED;
   if (s->profiling) s->prof.before(1, stream);
@@ -575,9 +574,8 @@ int moe_stack_device_error(moe_stack s, cudaStream_t stream) {
     if (cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess ||
         cudaMemset(s->amax, 0, static_cast<size_t>(s->L) * moe::kMaxDistinct * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(s->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
-        cudaMemset(s->logits, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.n_experts * 8) != cudaSuccess ||
-        cudaMemset(s->ypart, 0, s->ypart_bytes) != cudaSuccess ||
-        cudaMemset(s->ty, 0, moe::decode_ty_bytes(s->cfg.hidden)) != cudaSuccess ||
+        cudaMemset(s->tile_cnt, 0, static_cast<size_t>(s->cfg.hidden / 16) * 4) != cudaSuccess ||
+        cudaMemset(s->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.hidden * 8) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }

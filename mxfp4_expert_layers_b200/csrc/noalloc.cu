@@ -22,22 +22,18 @@ constexpr int kStaticMaxHidden = 4096;
 constexpr size_t kStaticH = static_cast<size_t>(kMaxDistinct) * kMaxTokGemv * kStaticMaxInter * sizeof(float);
 constexpr size_t kStaticAmax = 1024;     // >= kMaxDistinct * kMaxTokGemv unsigned
 constexpr size_t kStaticSync = 256;      // >= kSyncWords unsigned
-constexpr size_t kStaticTlog = static_cast<size_t>(kMaxTokGemv) * MOE_MAX_EXPERTS * sizeof(unsigned long long);
-constexpr int kStaticMaxCtas = 160;      // SMs of the device, at most
-// partial sums of y: 2 x R x (ceil(CTAs / R) + 2) x 4 tokens x 16 rows x 2
-// words, R = hidden / 16 <= 256, which is at most 2 x (CTAs + 3 R) x 128 words
-constexpr size_t kStaticYpart =
-    static_cast<size_t>(2) * (kStaticMaxCtas + 3 * (kStaticMaxHidden / 16)) * kMaxTokGemv * 16 * 2 * 8;
+constexpr size_t kStaticTile = static_cast<size_t>(kStaticMaxHidden / 16) * sizeof(unsigned);
+constexpr size_t kStaticYacc = static_cast<size_t>(kMaxTokGemv) * kStaticMaxHidden * sizeof(double);
 static_assert(kStaticAmax >= kMaxDistinct * kMaxTokGemv * sizeof(unsigned), "amax area");
 static_assert(kStaticSync >= kSyncWords * sizeof(unsigned), "counter area");
-// layout: h | amax | counters | tagged logits | error word | partial sums
-// of y (everything after h starts at zero)
+// layout: h | amax | counters | shared-row-tile counts | float64 row sums |
+// error word (everything after h starts at zero)
 constexpr size_t kOffAmax = kStaticH;
 constexpr size_t kOffSync = kOffAmax + kStaticAmax;
-constexpr size_t kOffTlog = kOffSync + kStaticSync;
-constexpr size_t kOffErr = kOffTlog + kStaticTlog;
-constexpr size_t kOffYpart = kOffErr + 256;
-constexpr size_t kStaticBytes = kOffYpart + kStaticYpart;
+constexpr size_t kOffTile = kOffSync + kStaticSync;
+constexpr size_t kOffYacc = kOffTile + kStaticTile;
+constexpr size_t kOffErr = kOffYacc + kStaticYacc;
+constexpr size_t kStaticBytes = kOffErr + 256;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 
@@ -103,7 +99,6 @@ extern "C" int moe_forward_static(const moe_config* cfg, const moe_weights* w, c
   int sms = 0, budget = 0;
   const int rc = scratch_for_current_device(&base, &sms, &budget);
   if (rc != MOE_OK) return rc;
-  if (sms > kStaticMaxCtas || decode_ypart_bytes(cfg->hidden, sms) > kStaticYpart) return MOE_ERR_UNSUPPORTED;
   DecodeArgs a{};
   a.H = cfg->hidden; a.I = cfg->inter; a.E = cfg->n_experts; a.k = cfg->top_k; a.n_shared = cfg->n_shared;
   a.T = T;
@@ -118,9 +113,9 @@ extern "C" int moe_forward_static(const moe_config* cfg, const moe_weights* w, c
   a.h = reinterpret_cast<float*>(base);
   a.amax = reinterpret_cast<unsigned*>(base + kOffAmax);
   a.sync = reinterpret_cast<unsigned*>(base + kOffSync);
-  a.tlogits = reinterpret_cast<unsigned long long*>(base + kOffTlog);
+  a.tile_cnt = reinterpret_cast<unsigned*>(base + kOffTile);
+  a.yacc = reinterpret_cast<double*>(base + kOffYacc);
   a.err = reinterpret_cast<int*>(base + kOffErr);
-  a.ypart = reinterpret_cast<unsigned long long*>(base + kOffYpart);
   a.y = y;
   if (!decode_plan(a, sms, budget)) return MOE_ERR_UNSUPPORTED;
   return launch_decode(a, sms, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
