@@ -127,6 +127,7 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int32_t
 #pragma unroll
   for (int m = 0; m < 16; ++m)
     if (key[m] > bk) { bk = key[m]; bm = m; }
+  MOE_TRACE_POINT(3, 19);
   unsigned my_key = 0;
   int my_id = -1;
   for (int r = 0; r < k; ++r) {
@@ -143,6 +144,7 @@ __device__ __forceinline__ void topk_warp(const float* lg, int E, int k, int32_t
     }
     if (lane == r) { my_key = best; my_id = id; }
   }
+  MOE_TRACE_POINT(3, 58);
   const float my_v = key_f32(my_key);
   const double top = static_cast<double>(__shfl_sync(0xffffffffu, my_v, 0));
   const double z = lane < k ? exp(static_cast<double>(my_v) - top) : 0.0;
@@ -420,7 +422,9 @@ decode_kernel(DecodeArgs a) {
       }
       ok = __syncthreads_and(ok);
       if (!ok) break;
+      MOE_TRACE_POINT(3, 17);
       if (kStack) residual_norm(a, rs, a.ybuf + static_cast<size_t>((l - 1) & 1) * T * H, xb, red_d, den_s);
+      MOE_TRACE_POINT(3, 18);
     }
     if (kDebug && a.dbg_x && cta == 0)
       for (int u = tid; u < T * H / 8; u += kThreads)
@@ -446,6 +450,7 @@ decode_kernel(DecodeArgs a) {
         if (lane == 0) red_f[warp][tt] = m;
       }
       __syncthreads();
+      MOE_TRACE_POINT(3, 56);
       if (tid < T) {
         float amax = 0.f;
         for (int i = 0; i < kWarps; ++i) amax = fmaxf(amax, red_f[i][tid]);
@@ -453,6 +458,7 @@ decode_kernel(DecodeArgs a) {
         if (kDebug && cta == 0 && a.dbg.xs) a.dbg.xs[tid] = xs[tid];
       }
       __syncthreads();
+      MOE_TRACE_POINT(3, 57);
       for (int u = tid; u < T * upr; u += kThreads) {
         const uint4 v = reinterpret_cast<const uint4*>(xb)[u];
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -508,8 +514,6 @@ decode_kernel(DecodeArgs a) {
       if (tid == 0) {
         __threadfence();
         red_release_add_u32(a.sync + kSyncRoute, 1u);
-        // the router rows are used: the next layer's stream in meanwhile
-        if (l + 1 < L && nr > 0 && ok) copy_in(sm.rr, lw_next.Wr + static_cast<size_t>(row0) * H, nr * H * 2, &fr, &ur);
         if (!poll_geq_bounded(a.sync + kSyncRoute, static_cast<unsigned>((l + 1) * G), a.err)) {
           ok = false;
           note_timeout(__LINE__, l, -1);
@@ -520,6 +524,7 @@ decode_kernel(DecodeArgs a) {
       MOE_TRACE_POINT(3, 4);
       if (warp < T) topk_warp(a.logits + static_cast<size_t>(warp) * E, E, a.k, s_ids + warp * a.k, s_w + warp * a.k);
       __syncthreads();
+      MOE_TRACE_POINT(3, 16);
       if (cta == 0) {
         if (tid < T * a.k) {
           if (ids_l) ids_l[tid] = s_ids[tid];
@@ -672,6 +677,9 @@ decode_kernel(DecodeArgs a) {
     if (tid == 0) {
       __threadfence();
       red_release_add_u32(a.sync + kSyncGU, 1u);
+      // the router rows of this layer are used: the next layer's stream in
+      // while the barrier is waited for (the wait hides the copy's issue)
+      if (a.route && l + 1 < L && nr > 0) copy_in(sm.rr, lw_next.Wr + static_cast<size_t>(row0) * H, nr * H * 2, &fr, &ur);
       if (!poll_geq_bounded(a.sync + kSyncGU, static_cast<unsigned>((l + 1) * G), a.err)) {
         ok = false;
         note_timeout(__LINE__, l, -1);
