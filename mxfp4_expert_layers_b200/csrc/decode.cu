@@ -85,19 +85,21 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool v) {
 
 // Wait for use `use` of a ring slot: first until its copy has been issued
 // (uses > use; another warp group may still be consuming the previous use),
-// then for the copy's bytes.  Bounded like every wait.
-__device__ __forceinline__ bool wait_slot(uint64_t* bar, const int* uses, int use, int* err) {
+// then for the copy's bytes.  Bounded like every wait; the loops are out of
+// line.
+__device__ __noinline__ bool wait_issued_slow(const int* uses, int use, int* err) {
   const volatile int* u = uses;
-  if (*u <= use) {
-    const unsigned long long t0 = global_ns();
-    for (long long i = 1;; ++i) {
-      if (*u > use) break;
-      if ((i & 255) == 0 && global_ns() - t0 > kWaitNs) {
-        if (err) atomicOr(err, kErrTimeout);
-        return false;
-      }
+  const unsigned long long t0 = global_ns();
+  for (long long i = 1;; ++i) {
+    if (*u > use) return true;
+    if ((i & 255) == 0 && global_ns() - t0 > kWaitNs) {
+      if (err) atomicOr(err, kErrTimeout);
+      return false;
     }
   }
+}
+__device__ __forceinline__ bool wait_slot(uint64_t* bar, const int* uses, int use, int* err) {
+  if (*reinterpret_cast<const volatile int*>(uses) <= use && !wait_issued_slow(uses, use, err)) return false;
   return mbar_wait_bounded(bar, use & 1, err);
 }
 

@@ -147,6 +147,37 @@ def test_gpu_quantize_rows_matches_oracle():
     assert np.array_equal(s.cpu().numpy(), rs)
 
 
+def test_gpu_quantize_near_code_boundaries_matches_oracle():
+    """The quotient v / s taken through its reciprocal: rows whose values sit
+    on, and within 12 float32 ulps of, every exact midpoint between adjacent
+    E4M3 values (and every E4M3 value) times a scale that is not a power of
+    two, both signs; the codes equal those of the correctly rounded float32
+    quotient."""
+    rng = np.random.default_rng(7)
+    vals = np.unique(np.abs(OF.e4m3_value(np.arange(0x7F))))
+    pts = np.concatenate([(vals[1:] + vals[:-1]) / 2, vals])
+    rows = []
+    for amax in rng.uniform(1e-3, 1e3, 24).astype(np.float32):
+        s = np.float32(amax / np.float32(448.0))
+        base = (pts * np.float64(s)).astype(np.float32)
+        near = (base.view(np.int32)[:, None] + np.arange(-12, 13, dtype=np.int32)[None, :]).ravel()
+        v = near.view(np.float32)
+        v = v[np.abs(v) < amax]
+        rows.append(np.concatenate([[amax], v, -v]).astype(np.float32))
+    cols = max(r.size for r in rows)
+    v = np.zeros((len(rows), cols), np.float32)
+    for i, r in enumerate(rows):
+        v[i, :r.size] = r
+    q = torch.empty(v.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(v.shape[0], dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8(to_dev(v), v.shape[0], v.shape[1], q, s)
+    rq, rs = OM.quantize_fp8(v)
+    assert np.array_equal(s.cpu().numpy(), rs)
+    got = q.cpu().numpy()
+    bad = np.argwhere(got != rq)
+    assert bad.size == 0, [(float(v[i, j]), int(got[i, j]), int(rq[i, j])) for i, j in bad[:8]]
+
+
 # --------------------------------------------------------------- routing --
 
 @pytest.mark.parametrize("E,T,bias", [(32, 1, False), (512, 1, False), (512, 4, False),
