@@ -210,6 +210,11 @@ __device__ __noinline__ void note_timeout(int line, int layer, int entry) {
 // CTA owning down slab q: the largest c with floor(c * S / G) <= q.
 __device__ __forceinline__ int slab_owner(int q, int S, int G) { return ((q + 1) * G + S - 1) / S - 1; }
 __device__ __forceinline__ int slab_start(int c, int S, int G) { return c * S / G; }
+// Row tile r of y takes the nd slabs r nd .. r nd + nd - 1; it is shared when
+// they lie in more than one CTA's range (Stot = (H/16) nd slabs over G CTAs).
+__device__ __forceinline__ bool tile_shared(int r, int nd, int Stot, int G) {
+  return nd > 0 && slab_owner(r * nd, Stot, G) != slab_owner(r * nd + nd - 1, Stot, G);
+}
 
 __device__ __forceinline__ LayerW layer_ptrs(const DecodeArgs& a, int l) {
   if (!a.layers) return a.layer0;
@@ -269,14 +274,30 @@ __device__ __forceinline__ void issue_dn(const DecodeArgs& a, const Smem& sm, co
 
 // Residual add and RMS normalisation of the stack (every CTA, same values):
 // r = bf16(r + y); x = bf16(r / sqrt(mean(r^2) + eps)), float64 arithmetic.
-// rs and xb are [T][H] bfloat16 in shared memory.
-__device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t* y, uint16_t* xb,
-                              double (*red)[kMaxTokGemv], double* den_s) {
+// rs and xb are [T][H] bfloat16 in shared memory.  The previous layer left
+// its y in two places: the row tiles one CTA finished, as bfloat16 in y; the
+// row tiles several CTAs added to (tile_shared with that layer's nd), as
+// float64 sums in ysum ([T][H]), rounded here the way the CTA finishing them
+// would have.
+__device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t* y, const double* ysum, int nd,
+                              uint16_t* xb, double (*red)[kMaxTokGemv], double* den_s) {
   const int H = a.H, T = a.T, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int upr = H / 8;
+  const int upr = H / 8, Stot = (H / 16) * nd, G = gridDim.x;
   double ss[kMaxTokGemv] = {0.0, 0.0, 0.0, 0.0};
   for (int u = tid; u < T * upr; u += kThreads) {
-    const uint4 yv = __ldcg(reinterpret_cast<const uint4*>(y) + u);
+    uint4 yv;
+    if (tile_shared((u % upr) >> 1, nd, Stot, G)) {
+      const double2* p = reinterpret_cast<const double2*>(ysum + static_cast<size_t>(u / upr) * H + 8 * (u % upr));
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double2 v = __ldcg(p + j);
+        w[j] = static_cast<uint32_t>(f64_to_bf16_rne(v.x)) | (static_cast<uint32_t>(f64_to_bf16_rne(v.y)) << 16);
+      }
+      yv = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      yv = __ldcg(reinterpret_cast<const uint4*>(y) + u);
+    }
     const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
     const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
@@ -402,6 +423,10 @@ decode_kernel(DecodeArgs a) {
   }
   if (warp < min(ns, NG) && lane == 0) issue_gu(a, sm, lw, dist.expert, warp, warp);
   int npre = min(ns, NG);  // gate/up tiles of the coming layer already in flight
+  // the previous layer's distinct-expert count and the row tiles this CTA
+  // added to there (stack: their float64 sums are zeroed once read)
+  int nd_prev = 0;
+  int zsh[2] = {-1, -1};
   int gu_base = 0, dn_base = 0;
 
   pdl_wait();
@@ -425,7 +450,9 @@ decode_kernel(DecodeArgs a) {
       ok = __syncthreads_and(ok);
       if (!ok) break;
       MOE_TRACE_POINT(3, 17);
-      if (kStack) residual_norm(a, rs, a.ybuf + static_cast<size_t>((l - 1) & 1) * T * H, xb, red_d, den_s);
+      if (kStack)
+        residual_norm(a, rs, a.ybuf + static_cast<size_t>((l - 1) & 1) * T * H,
+                      a.yacc + static_cast<size_t>((l - 1) & 1) * kMaxTokGemv * H, nd_prev, xb, red_d, den_s);
       MOE_TRACE_POINT(3, 18);
     }
     if (kDebug && a.dbg_x && cta == 0)
@@ -690,8 +717,22 @@ decode_kernel(DecodeArgs a) {
     ok = __syncthreads_and(ok);
     if (!ok) break;
     MOE_TRACE_POINT(3, 8);
+    if (stack && tid < 16 * T) {
+      // every CTA has read the previous layer's sums (its residual step came
+      // before both barriers since): zero the tiles this CTA added to, for
+      // the layer after this one
+      double* ysum = a.yacc + static_cast<size_t>((l - 1) & 1) * kMaxTokGemv * H;
+      for (int i = 0; i < 2; ++i)
+        if (zsh[i] >= 0) ysum[static_cast<size_t>(tid % T) * H + 16 * zsh[i] + tid / T] = 0.0;
+    }
+    zsh[0] = zsh[1] = -1;
 
     // ---- 4. down + combine: group grp takes slabs grp, grp + 4, ...
+    // stack at one token: row tiles shared between CTAs are left as float64
+    // sums for the next layer's residual step to round (no hand-off between
+    // CTAs here); at more tokens that step would read four times the bytes,
+    // so the last CTA to add rounds them as in a single layer
+    const bool defer = stack && T == 1;
     uint16_t* y_l = (!stack && l == L - 1) ? a.y : a.ybuf + static_cast<size_t>(l & 1) * T * H;
     // a part of a layer split over GPUs: its float32 part of y (not rounded)
     float* y32_l = (!stack && l == L - 1) ? a.y32 : nullptr;
@@ -848,8 +889,10 @@ decode_kernel(DecodeArgs a) {
       MOE_TRACE_POINT(3, 10);
       // finish the CTA's row tiles: owned ones directly; the first and last,
       // when shared with a neighbouring CTA, through the float64 accumulators
-      // (whichever CTA adds last rounds them)
+      // (deferred: read and rounded by every CTA in the next layer's residual
+      // step; otherwise whichever CTA adds last rounds them)
       const int nrt = ok ? (q1 - 1) / nd - rt0 + 1 : 0;
+      double* yacc_l = a.yacc + (defer ? static_cast<size_t>(l & 1) * kMaxTokGemv * H : 0);
       const int row = tid / T, tt = tid % T;
       int shared_lr[2] = {-1, -1};
       int nsh = 0;
@@ -865,7 +908,7 @@ decode_kernel(DecodeArgs a) {
             acc += v;
             v = 0.0;
           }
-          if (!owned) atomicAdd(a.yacc + yi, acc);
+          if (!owned) atomicAdd(yacc_l + yi, acc);
           else if (y32_l) y32_l[yi] = static_cast<float>(acc);
           else y_l[yi] = f64_to_bf16_rne(acc);
         }
@@ -875,7 +918,11 @@ decode_kernel(DecodeArgs a) {
           ++nsh;
         }
       }
-      if (nsh > 0) {
+      if (defer) {
+        // the sums stay in yacc_l for the next layer's residual step
+        zsh[0] = nsh > 0 ? rt0 + shared_lr[0] : -1;
+        zsh[1] = nsh > 1 ? rt0 + shared_lr[1] : -1;
+      } else if (nsh > 0) {
         __syncthreads();
         if (tid == 0) {
           __threadfence();
@@ -897,16 +944,17 @@ decode_kernel(DecodeArgs a) {
           const int r = rt0 + shared_lr[i];
           if (tid < 16 * T) {
             const size_t yi = static_cast<size_t>(tt) * H + 16 * r + row;
-            const double v = __ldcg(a.yacc + yi);
+            const double v = __ldcg(yacc_l + yi);
             if (y32_l) y32_l[yi] = static_cast<float>(v);
             else y_l[yi] = f64_to_bf16_rne(v);
-            a.yacc[yi] = 0.0;
+            yacc_l[yi] = 0.0;
           }
           if (tid == 0) a.tile_cnt[r] = 0u;
         }
       }
     }
     dn_base += nq;
+    nd_prev = defer ? nd : 0;
     MOE_TRACE_POINT(3, 11);
     // ---- 5. y of this layer complete (for the next layer or the final norm)
     __syncthreads();
@@ -923,7 +971,14 @@ decode_kernel(DecodeArgs a) {
       note_timeout(__LINE__, L, -1);
     }
     if (__syncthreads_and(ok)) {
-      residual_norm(a, rs, a.ybuf + static_cast<size_t>((L - 1) & 1) * T * H, xb, red_d, den_s);
+      double* ysum = a.yacc + static_cast<size_t>((L - 1) & 1) * kMaxTokGemv * H;
+      residual_norm(a, rs, a.ybuf + static_cast<size_t>((L - 1) & 1) * T * H, ysum, nd_prev, xb, red_d, den_s);
+      // the last layer's sums are read: zero them for the next call
+      const int Stot = (H / 16) * nd_prev;
+      for (int i = tid; i < (H / 16) * 16 * T; i += kThreads) {
+        const int r = i / (16 * T);
+        if (tile_shared(r, nd_prev, Stot, G)) ysum[static_cast<size_t>(i % T) * H + 16 * r + (i / T) % 16] = 0.0;
+      }
       for (int u = tid; u < T * H / 8; u += kThreads) {
         reinterpret_cast<uint4*>(a.r_io)[u] = reinterpret_cast<const uint4*>(rs)[u];
         reinterpret_cast<uint4*>(a.x_io)[u] = reinterpret_cast<const uint4*>(xb)[u];

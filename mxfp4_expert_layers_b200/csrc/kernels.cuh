@@ -80,7 +80,7 @@ struct DecodeArgs {
   unsigned* amax;       // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;       // [kSyncWords]
   unsigned* tile_cnt;   // [H/16]
-  double* yacc;         // [kMaxTokGemv][H]
+  double* yacc;         // [kMaxTokGemv][H]; stack: [2][kMaxTokGemv][H], by layer parity
   uint16_t* ybuf;       // [2][T][H] y of stacked layers
   int* err;
   moe_debug dbg;        // plain layer only

@@ -461,7 +461,7 @@ struct moe_stack_s {
   unsigned* amax;        // [L][kMaxDistinct][kMaxTokGemv]
   unsigned* sync;
   unsigned* tile_cnt;
-  double* yacc;
+  double* yacc;          // [2][kMaxTokGemv][H] float64 sums of the shared row tiles, by layer parity
   uint16_t* ybuf;        // [2][kMaxTokGemv][H] y of the stacked layers
   int* err;
   int n_sms;
@@ -497,7 +497,7 @@ int moe_stack_create(const moe_handle* layers, int n_layers, moe_stack* out) {
   const size_t n_amax = up256(static_cast<size_t>(n_layers) * moe::kMaxDistinct * moe::kMaxTokGemv * 4);
   const size_t n_sync = up256(static_cast<size_t>(moe::kSyncWords) * 4);
   const size_t n_tcnt = up256(static_cast<size_t>(c.hidden / 16) * 4);
-  const size_t n_yacc = up256(static_cast<size_t>(moe::kMaxTokGemv) * c.hidden * 8);
+  const size_t n_yacc = up256(static_cast<size_t>(2) * moe::kMaxTokGemv * c.hidden * 8);  // by layer parity
   const size_t n_ybuf = n_tcnt + n_yacc + up256(static_cast<size_t>(2) * moe::kMaxTokGemv * c.hidden * 2);
   const size_t n_err = 256;
   const size_t bytes = n_layers_b + n_logits + n_h + n_amax + n_sync + n_ybuf + n_err;
@@ -575,7 +575,7 @@ int moe_stack_device_error(moe_stack s, cudaStream_t stream) {
         cudaMemset(s->amax, 0, static_cast<size_t>(s->L) * moe::kMaxDistinct * moe::kMaxTokGemv * 4) != cudaSuccess ||
         cudaMemset(s->sync, 0, static_cast<size_t>(moe::kSyncWords) * 4) != cudaSuccess ||
         cudaMemset(s->tile_cnt, 0, static_cast<size_t>(s->cfg.hidden / 16) * 4) != cudaSuccess ||
-        cudaMemset(s->yacc, 0, static_cast<size_t>(moe::kMaxTokGemv) * s->cfg.hidden * 8) != cudaSuccess ||
+        cudaMemset(s->yacc, 0, static_cast<size_t>(2) * moe::kMaxTokGemv * s->cfg.hidden * 8) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return MOE_ERR_CUDA;
   }
