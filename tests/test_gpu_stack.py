@@ -136,6 +136,30 @@ def test_gpu_stack_matches_oracle_teacher_forced_e512(T):
             ly.close()
 
 
+def test_gpu_stack_token_counts_interleaved():
+    """One stack object called at 1, 4, 1, 2 and 1 tokens in turn (E = 512,
+    H = 2560: at one token the row tiles two CTAs share are left as two parts
+    for the next layer; at more tokens they are summed into accumulators that
+    must be zero again after every call): each call equals one moe_decode +
+    one moe_residual_rmsnorm per layer."""
+    layers = [GpuLayer(0, 120 + l, 512, bias=True) for l in range(2)]
+    st = moe.moe_stack_create([ly.handle for ly in layers])
+    try:
+        for i, T in enumerate((1, 4, 1, 2, 1)):
+            x0 = synth.hidden_states(0, 9000 + i, T, H0)
+            r, x = to_dev_u16(x0), to_dev_u16(x0)
+            moe.moe_stack_decode(st, r, x, T, EPS, None, None, None)
+            torch.cuda.synchronize()
+            assert moe.moe_stack_device_error(st) == moe.MOE_OK
+            ref = _layer_by_layer(layers, x0)
+            assert np.array_equal(u16(r), ref[0]), (i, T)
+            assert np.array_equal(u16(x), ref[1]), (i, T)
+    finally:
+        moe.moe_stack_destroy(st)
+        for ly in layers:
+            ly.close()
+
+
 def test_gpu_stack_repeats_and_single_layer():
     """Back-to-back calls give the same result; a one-layer stack equals
     moe_decode followed by moe_residual_rmsnorm."""
