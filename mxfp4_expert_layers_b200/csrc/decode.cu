@@ -14,8 +14,8 @@
 //
 // One CTA per SM, 16 warps in 4 groups of 4.  A CTA streams its share of a
 // layer through shared memory with 1-D bulk copies: its slice of router rows
-// (own region, the next layer's rows prefetched as soon as the current ones
-// are used), its gate/up tiles (a ring of NG fixed slots) and its down slabs
+// (own region; the next layer's rows are fetched while the gate/up hand-off
+// is waited for), its gate/up tiles (a ring of NG fixed slots) and its down slabs
 // (a ring of ND slots).  Entry j of a ring lives in slot j mod N; the group
 // that consumes entry j refills the slot with entry j + N, so no thread
 // coordinates the copies.
@@ -40,8 +40,12 @@
 //     slabs goes to group i mod 4, the routing weight and h scale folded
 //     into the float64 epilogue.  Row tiles the CTA owns are rounded to
 //     bfloat16 directly; a row tile shared with a neighbouring CTA is summed
-//     in a float64 accumulator and rounded by whichever CTA adds last.
+//     in a float64 accumulator and rounded by whichever CTA adds last, or,
+//     in a stack at one token, by every CTA of the next layer as it reads y.
 //  5. a grid-wide arrive marks y complete for the next layer.
+//
+// A call may hold only the routed experts ep_lo .. ep_hi-1 (the layer split
+// over several GPUs); it then writes its float32 part of y.
 //
 // Every wait is bounded (one second of %globaltimer) and records
 // kErrTimeout; a CTA that gave up lets its copies in flight land and exits.
