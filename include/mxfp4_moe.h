@@ -178,7 +178,7 @@ int moe_decode(moe_handle h, const uint16_t* x, int T, int32_t* topk_ids, float*
  * device) -- and so cannot call moe_create, which allocates a workspace.
  * The experts run exactly as in moe_forward (same kernel and results), with
  * their scratch memory (SwiGLU outputs, per-expert amax, counters, the
- * launch counter and tagged logits: about 575 KB) in one fixed array inside
+ * shared-row-tile counters and float64 row sums: about 691 KB) in one fixed array inside
  * this library, which every GPU that loads the library keeps until the
  * process exits.
  *   - Limits: T in 1..MOE_GEMV_MAX_TOKENS, inter <= 1024 and hidden <= 4096;
