@@ -131,6 +131,23 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
   return r;
 }
 
+// bfloat16 bits (round to nearest even) of q = RN(r * inv), where
+// inv = RN(1 / den) stands in for a division by den: q is within 2 ulps of
+// r / den, so it rounds like the quotient unless it lies within 8 ulps of a
+// midpoint between two bfloat16 values (the 45 fraction bits below the
+// bfloat16 ones near 2^44) or outside the normal bfloat16 range (zero
+// excepted); then slow is set and the caller divides.
+__device__ __forceinline__ uint16_t bf16_of_product(double r, double inv, bool& slow) {
+  const double q = r * inv;
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(q));
+  const unsigned long long low = b & ((1ull << 45) - 1ull);
+  const unsigned ex = static_cast<unsigned>(b >> 52) & 0x7FFu;
+  const bool safe = (ex >= 897u && ex < 0x47Fu && (low + 8ull < (1ull << 44) || low > (1ull << 44) + 8ull)) ||
+                    (b << 1) == 0ull;  // +-0 = +-0 / den
+  slow |= !safe;
+  return f64_to_bf16_rne(q);
+}
+
 // ------------------------------------------------------------- reductions --
 __device__ __forceinline__ double warp_sum_f64(double v, int width = 32) {
   for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, width);

@@ -335,19 +335,32 @@ __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t*
     double s = 0.0;
     for (int w = 0; w < kWarps; ++w) s += red[w][tid];
     den_s[tid] = sqrt(s / static_cast<double>(H) + static_cast<double>(a.eps));
+    den_s[kMaxTokGemv + tid] = 1.0 / den_s[tid];
   }
   __syncthreads();
   for (int u = tid; u < T * upr; u += kThreads) {
     const uint4 rv = reinterpret_cast<const uint4*>(rs)[u];
     const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-    const double den = den_s[u / upr];
+    // x = bf16(r / den) through the reciprocal, by division only where the
+    // two could round differently (bf16_of_product)
+    const double den = den_s[u / upr], inv = den_s[kMaxTokGemv + u / upr];
     uint32_t o[4];
+    bool slow = false;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float r0, r1;
       bf16x2_f32(rw[j], r0, r1);
-      o[j] = static_cast<uint32_t>(f64_to_bf16_rne(static_cast<double>(r0) / den)) |
-             (static_cast<uint32_t>(f64_to_bf16_rne(static_cast<double>(r1) / den)) << 16);
+      o[j] = static_cast<uint32_t>(bf16_of_product(r0, inv, slow)) |
+             (static_cast<uint32_t>(bf16_of_product(r1, inv, slow)) << 16);
+    }
+    if (slow) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float r0, r1;
+        bf16x2_f32(rw[j], r0, r1);
+        o[j] = static_cast<uint32_t>(f64_to_bf16_rne(static_cast<double>(r0) / den)) |
+               (static_cast<uint32_t>(f64_to_bf16_rne(static_cast<double>(r1) / den)) << 16);
+      }
     }
     reinterpret_cast<uint4*>(xb)[u] = make_uint4(o[0], o[1], o[2], o[3]);
   }
@@ -378,7 +391,7 @@ decode_kernel(DecodeArgs a) {
   __shared__ float xs[kMaxTokGemv];
   __shared__ float red_f[kWarps][kMaxTokGemv];
   __shared__ double red_d[kWarps][kMaxTokGemv];
-  __shared__ double den_s[kMaxTokGemv];
+  __shared__ double den_s[2 * kMaxTokGemv];  // RMS denominator, then its reciprocal
   __shared__ int s_abort;
   __shared__ int s_flag;
   __shared__ int s_last[2];
