@@ -233,6 +233,24 @@ def test_gpu_forward_small_shapes(T, n_shared, mode):
         L.close()
 
 
+@pytest.mark.parametrize("T", [1, 4])
+def test_gpu_forward_other_shape(T):
+    """A second shape set through the same kernels (the shapes are run-time
+    arguments): hidden 4096, expert width 1536, E = 32 top-8 + 1 shared, at one
+    and at four tokens, against the oracle."""
+    H, I = 4096, 1536
+    L = GpuLayer(5, 7, 32, H, I)
+    try:
+        for step in range(2):
+            x = synth.hidden_states(5, 70 + 10 * T + step, T, H)
+            ids, w, counts, y, dbg = _run(L, x, mode="fused")
+            ref = _oracle(L, x)
+            check_route(ids, w, counts, ref)
+            check_forward(y, dbg, ref)
+    finally:
+        L.close()
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_gpu_forward_config0_single_token(mode):
     """One token, E = 32 routed top-8 + 1 shared, H 2560, I 768, seed 0."""
