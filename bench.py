@@ -69,8 +69,8 @@ def parse():
 # changed since makes the figure stale: the line then reports traffic null.
 NCU_TRAFFIC = {
     # decode_kernel, 2-layer stack at T = 1, per layer (traffic grows with the layers a launch runs)
-    "decode_kernel": {"bytes": (61.837824e6 + 0.451072e6) / 2, "per": "layer",
-                      "src": "mxfp4_expert_layers_b200/csrc/decode.cu", "sha16": "82a7d191721ea994"},
+    "decode_kernel": {"bytes": (61.842432e6 + 0.805632e6) / 2, "per": "layer",
+                      "src": "mxfp4_expert_layers_b200/csrc/decode.cu", "sha16": "94d672980f03b8a0"},
     # tc_gemm_kernel<0> + tc_gemm_kernel<1> of one 512-token prefill call (Zipf routing)
     "tc_gemm_kernel": {"bytes": 228.321024e6 + 11.817728e6 + 116.868352e6 + 3.162112e6, "per": "call",
                        "src": "mxfp4_expert_layers_b200/csrc/prefill_tc.cu", "sha16": "7eabad916cda2413"},

@@ -284,10 +284,12 @@ __device__ __forceinline__ void issue_dn(const DecodeArgs& a, const Smem& sm, co
 // float64 sums in ysum ([T][H]), rounded here the way the CTA finishing them
 // would have.
 __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t* y, const double* ysum, int nd,
-                              uint16_t* xb, double (*red)[kMaxTokGemv], double* den_s) {
+                              uint16_t* xb, double (*red)[kMaxTokGemv], double* den_s, float* xs = nullptr,
+                              float (*red_f)[kMaxTokGemv] = nullptr) {
   const int H = a.H, T = a.T, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int upr = H / 8, Stot = (H / 16) * nd, G = gridDim.x;
   double ss[kMaxTokGemv] = {0.0, 0.0, 0.0, 0.0};
+  float mr[kMaxTokGemv] = {0.f, 0.f, 0.f, 0.f};
   for (int u = tid; u < T * upr; u += kThreads) {
     uint4 yv;
     if (tile_shared((u % upr) >> 1, nd, Stot, G)) {
@@ -307,6 +309,7 @@ __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t*
     const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
     uint32_t o[4];
     double part = 0.0;
+    float m = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float r0, r1, y0, y1;
@@ -315,27 +318,47 @@ __device__ void residual_norm(const DecodeArgs& a, uint16_t* rs, const uint16_t*
       const uint16_t s0 = f64_to_bf16_rne(static_cast<double>(r0) + static_cast<double>(y0));
       const uint16_t s1 = f64_to_bf16_rne(static_cast<double>(r1) + static_cast<double>(y1));
       o[j] = static_cast<uint32_t>(s0) | (static_cast<uint32_t>(s1) << 16);
-      const double q0 = bf16_bits_to_f32(s0), q1 = bf16_bits_to_f32(s1);
+      const float f0 = bf16_bits_to_f32(s0), f1 = bf16_bits_to_f32(s1);
+      const double q0 = f0, q1 = f1;
       part = fma(q0, q0, part);
       part = fma(q1, q1, part);
+      m = fmaxf(m, fmaxf(fabsf(f0), fabsf(f1)));
     }
     reinterpret_cast<uint4*>(rs)[u] = make_uint4(o[0], o[1], o[2], o[3]);
     const int t = u / upr;
 #pragma unroll
     for (int tt = 0; tt < kMaxTokGemv; ++tt)
-      if (tt == t) ss[tt] += part;
+      if (tt == t) {
+        ss[tt] += part;
+        mr[tt] = fmaxf(mr[tt], m);
+      }
   }
 #pragma unroll
   for (int tt = 0; tt < kMaxTokGemv; ++tt) {
     const double v = warp_sum_f64(ss[tt]);
-    if (lane == 0) red[warp][tt] = v;
+    const float mv = warp_max_f32(mr[tt]);
+    if (lane == 0) {
+      red[warp][tt] = v;
+      if (xs) red_f[warp][tt] = mv;
+    }
   }
   __syncthreads();
   if (tid < T) {
     double s = 0.0;
     for (int w = 0; w < kWarps; ++w) s += red[w][tid];
-    den_s[tid] = sqrt(s / static_cast<double>(H) + static_cast<double>(a.eps));
-    den_s[kMaxTokGemv + tid] = 1.0 / den_s[tid];
+    const double den = sqrt(s / static_cast<double>(H) + static_cast<double>(a.eps));
+    den_s[tid] = den;
+    den_s[kMaxTokGemv + tid] = 1.0 / den;
+    if (xs) {
+      // the x scale: max|x| = bf16(max|r| / den) (the division by den > 0 and
+      // the rounding keep the order); NaN there means the x are all NaN or
+      // the largest r is infinite, where a max over the x would give 0
+      float mx = 0.f;
+      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red_f[w][tid]);
+      float amax = bf16_bits_to_f32(f64_to_bf16_rne(static_cast<double>(mx) / den));
+      if (isnan(amax)) amax = 0.f;
+      xs[tid] = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+    }
   }
   __syncthreads();
   for (int u = tid; u < T * upr; u += kThreads) {
@@ -469,7 +492,8 @@ decode_kernel(DecodeArgs a) {
       MOE_TRACE_POINT(3, 17);
       if (kStack)
         residual_norm(a, rs, a.ybuf + static_cast<size_t>((l - 1) & 1) * T * H,
-                      a.yacc + static_cast<size_t>((l - 1) & 1) * kMaxTokGemv * H, nd_prev, xb, red_d, den_s);
+                      a.yacc + static_cast<size_t>((l - 1) & 1) * kMaxTokGemv * H, nd_prev, xb, red_d, den_s, xs,
+                      red_f);
       MOE_TRACE_POINT(3, 18);
     }
     if (kDebug && a.dbg_x && cta == 0)
@@ -477,6 +501,7 @@ decode_kernel(DecodeArgs a) {
         reinterpret_cast<uint4*>(a.dbg_x + static_cast<size_t>(l) * T * H)[u] = reinterpret_cast<const uint4*>(xb)[u];
     {
       const int upr = H / 8;
+      if (!(kStack && l > 0)) {  // a stacked layer's residual step set xs
       float mx[kMaxTokGemv] = {0.f, 0.f, 0.f, 0.f};
       for (int u = tid; u < T * upr; u += kThreads) {
         const uint4 v = reinterpret_cast<const uint4*>(xb)[u];
@@ -501,9 +526,10 @@ decode_kernel(DecodeArgs a) {
         float amax = 0.f;
         for (int i = 0; i < kWarps; ++i) amax = fmaxf(amax, red_f[i][tid]);
         xs[tid] = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-        if (kDebug && cta == 0 && a.dbg.xs) a.dbg.xs[tid] = xs[tid];
       }
       __syncthreads();
+      }
+      if (kDebug && cta == 0 && a.dbg.xs && tid < T) a.dbg.xs[tid] = xs[tid];
       MOE_TRACE_POINT(3, 57);
       for (int u = tid; u < T * upr; u += kThreads) {
         const uint4 v = reinterpret_cast<const uint4*>(xb)[u];
